@@ -1,0 +1,353 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle.
+
+Each test fixes the oracle to a closed form, a hand-worked golden fixture,
+an invariant the method notes state, or an independent library routine, so
+that a plausible slip in the oracle (a dropped term, a wrong sign, an
+off-by-one shift, a transposed operand, a wrong GQA mapping, >= for >) fails
+at least one of them.  No GPU is needed.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(7)
+
+
+# ---------------------------------------------------------------- RoPE (R1)
+def test_rope_position_zero_is_identity():
+    x = rng.standard_normal((3, 2, 8))
+    np.testing.assert_array_equal(O.rope(x, [0, 0, 0], 1e4), x)
+
+
+def test_rope_d2_closed_form():
+    # d = 2: one pair (x0, x1), inv_freq = theta^0 = 1, angle = pos.
+    for pos in (1, 2, 7):
+        y = O.rope(np.array([[[1.0, 0.0]]]), [pos], 123.0)[0, 0]
+        np.testing.assert_allclose(y, [math.cos(pos), math.sin(pos)], rtol=0, atol=1e-15)
+        y = O.rope(np.array([[[0.0, 1.0]]]), [pos], 123.0)[0, 0]
+        np.testing.assert_allclose(y, [-math.sin(pos), math.cos(pos)], rtol=0, atol=1e-15)
+
+
+def test_rope_half_split_pairing():
+    # d = 4, theta = 1e4: inv_freq = [1, 1e-2].  Element 1 pairs with element
+    # 3 at frequency 1e-2 (half split), not with element 0 (adjacent pairs).
+    x = np.zeros((1, 1, 4))
+    x[0, 0, 1] = 1.0
+    y = O.rope(x, [100], 1e4)[0, 0]
+    np.testing.assert_allclose(y, [0.0, math.cos(1.0), 0.0, math.sin(1.0)], atol=1e-13)
+
+
+def test_rope_matches_complex_rotation():
+    # Independent formulation: z_j = x_j + i x_{j+d/2} multiplied by e^{i a_j}.
+    d, theta = 16, 1e6
+    x = rng.standard_normal((5, 3, d))
+    pos = np.array([0, 3, 31, 1000, 32767])
+    y = O.rope(x, pos, theta)
+    a = pos[:, None] * (theta ** (-np.arange(d // 2) * 2.0 / d))[None, :]
+    z = (x[..., : d // 2] + 1j * x[..., d // 2:]) * np.exp(1j * a)[:, None, :]
+    np.testing.assert_allclose(y[..., : d // 2], z.real, atol=1e-12)
+    np.testing.assert_allclose(y[..., d // 2:], z.imag, atol=1e-12)
+
+
+def test_rope_relative_position_and_norm():
+    d = 32
+    q = rng.standard_normal((1, 1, d))
+    k = rng.standard_normal((1, 1, d))
+    a = (O.rope(q, [40], 1e4) * O.rope(k, [7], 1e4)).sum()
+    b = (O.rope(q, [540], 1e4) * O.rope(k, [507], 1e4)).sum()
+    assert abs(a - b) < 1e-10
+    np.testing.assert_allclose(np.linalg.norm(O.rope(q, [12345], 1e6)), np.linalg.norm(q), rtol=1e-14)
+
+
+# ---------------------------------------------------------- attention (R2)
+def test_attention_two_key_closed_form():
+    # d = 4 (scale 1/2): scores ln 3 and 0 -> weights 3/4 and 1/4.
+    q = np.array([[[2 * math.log(3.0), 0, 0, 0]]])
+    k = np.array([[[1.0, 0, 0, 0]], [[0.0, 0, 0, 0]]])
+    v = np.array([[[4.0, 0, 8, -4]], [[0.0, 4, 0, 4]]])
+    np.testing.assert_allclose(O.attention(q, k, v)[0, 0], [3.0, 1.0, 6.0, -2.0], atol=1e-14)
+
+
+def test_attention_single_key_and_uniform():
+    q = rng.standard_normal((3, 2, 8))
+    k = rng.standard_normal((1, 1, 8))
+    v = rng.standard_normal((1, 1, 8))
+    np.testing.assert_allclose(O.attention(q, k, v), np.broadcast_to(v[0, 0], (3, 2, 8)), atol=1e-15)
+    k = rng.standard_normal((5, 1, 8))
+    v = rng.standard_normal((5, 1, 8))
+    np.testing.assert_allclose(O.attention(np.zeros((1, 1, 8)), k, v)[0, 0], v[:, 0].mean(0), atol=1e-15)
+
+
+def test_attention_gqa_contiguous_groups():
+    # Hq=4, Hkv=2: heads 0,1 read kv head 0 (values 1), heads 2,3 kv head 1 (values 2).
+    q = rng.standard_normal((2, 4, 8))
+    k = rng.standard_normal((3, 2, 8))
+    v = np.zeros((3, 2, 8))
+    v[:, 0] = 1.0
+    v[:, 1] = 2.0
+    o = O.attention(q, k, v)
+    np.testing.assert_allclose(o[:, 0:2], 1.0, atol=1e-15)
+    np.testing.assert_allclose(o[:, 2:4], 2.0, atol=1e-15)
+
+
+def test_attention_matches_scipy_softmax():
+    q = rng.standard_normal((4, 2, 8))
+    k = rng.standard_normal((6, 1, 8))
+    v = rng.standard_normal((6, 1, 8))
+    allowed = rng.random((4, 6)) < 0.6
+    allowed[:, 0] = True
+    o = O.attention(q, k, v, allowed)
+    for h in range(2):
+        s = q[:, h] @ k[:, 0].T / math.sqrt(8)
+        s[~allowed] = -np.inf
+        np.testing.assert_allclose(o[:, h], scipy.special.softmax(s, axis=1) @ v[:, 0], atol=1e-14)
+
+
+def test_attention_key_permutation_invariance():
+    q = rng.standard_normal((4, 2, 8))
+    k = rng.standard_normal((9, 1, 8))
+    v = rng.standard_normal((9, 1, 8))
+    p = rng.permutation(9)
+    np.testing.assert_allclose(O.attention(q, k, v), O.attention(q, k[p], v[p]), atol=1e-14)
+
+
+# ----------------------------------------- block cache == full recompute (R3)
+def _seq(T, Hq, Hkv, d, seed):
+    r = np.random.default_rng(seed)
+    return (r.standard_normal((T, Hq, d)), r.standard_normal((T, Hkv, d)), r.standard_normal((T, Hkv, d)))
+
+
+@pytest.mark.parametrize("n_prev", [0, 1, 3])
+def test_cached_block_equals_full_recompute(n_prev):
+    # Finished blocks never see later ones, so their keys are reusable like an
+    # autoregressive KV cache ([N1] key design 3, [N4] hierarchical cache): the
+    # cached decode of block n_prev equals recomputing the whole sequence under
+    # the block-causal mask.
+    D, Hq, Hkv, d, theta = 32, 4, 2, 16, 1e4
+    T = D * (n_prev + 1)
+    q, k, v = _seq(T, Hq, Hkv, d, 11 + n_prev)
+    cache = O.OracleCache(1, Hkv, d, theta)
+    for b in range(n_prev):
+        cache.commit(0, k[b * D:(b + 1) * D], v[b * D:(b + 1) * D])
+    got = O.block_attn_seq(cache.k[0], cache.v[0], q[-D:], k[-D:], v[-D:], theta)
+    want = O.full_sequence_attn(q, k, v, theta, D, rows=np.arange(T - D, T))
+    np.testing.assert_allclose(got, want, atol=1e-12)
+
+
+def test_commit_one_at_a_time_equals_together():
+    D, Hkv, d, theta = 32, 2, 8, 1e6
+    _, k, v = _seq(4 * D, 2, Hkv, d, 5)
+    a = O.OracleCache(1, Hkv, d, theta)
+    for b in range(4):
+        a.commit(0, k[b * D:(b + 1) * D], v[b * D:(b + 1) * D])
+    b_ = O.OracleCache(1, Hkv, d, theta)
+    b_.commit(0, k, v)
+    np.testing.assert_array_equal(a.k[0], b_.k[0])
+    np.testing.assert_array_equal(a.v[0], b_.v[0])
+
+
+def test_empty_prefix_is_plain_bidirectional_attention():
+    D, Hq, Hkv, d, theta = 32, 4, 2, 8, 1e4
+    q, k, v = _seq(D, Hq, Hkv, d, 3)
+    got = O.block_attn_seq(np.zeros((0, Hkv, d)), np.zeros((0, Hkv, d)), q, k, v, theta)
+    pos = np.arange(D)
+    want = O.attention(O.rope(q, pos, theta), O.rope(k, pos, theta), v)
+    np.testing.assert_allclose(got, want, atol=1e-14)
+
+
+def test_block_causal_allowed_pattern():
+    a = O.block_causal_allowed(8, 8, 4)
+    assert a[0, 3] and not a[0, 4] and a[4, 0] and a[5, 7] and a[7, 4]
+
+
+# ------------------------------------------------ 2L x 2L mixed mask (R4)
+def test_mixed_mask_golden_L8_D4():
+    rows = [ln.strip() for ln in open(os.path.join(GOLDEN, "mixed_mask_L8_D4.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    want = np.array([[c == "1" for c in r] for r in rows])
+    np.testing.assert_array_equal(O.mixed_mask(8, 4), want)
+
+
+@pytest.mark.parametrize("L,D", [(64, 8), (64, 32), (2048, 32)])
+def test_mixed_mask_pair_count_closed_form(L, D):
+    # B = L/D blocks: noisy->noisy L*D, noisy->clean D^2 B(B-1)/2,
+    # clean->clean D^2 B(B+1)/2.  At L=2048, D=32: 4,259,840 pairs.
+    B = L // D
+    want = L * D + D * D * B * (B - 1) // 2 + D * D * B * (B + 1) // 2
+    A = O.mixed_mask(L, D)
+    assert int(A.sum()) == want
+    if (L, D) == (2048, 32):
+        assert want == 4_259_840
+    assert A.any(axis=1).all()          # every query row sees at least one key
+
+
+def test_mask_attn_clean_rows_equal_block_causal_of_x0():
+    L, D, Hq, Hkv, d = 64, 8, 4, 2, 8
+    r = np.random.default_rng(9)
+    q, k, v = (r.standard_normal((1, 2 * L, h, d)) for h in (Hq, Hkv, Hkv))
+    got = O.mask_attn(q, k, v, L, D, rows=np.arange(L, 2 * L))[0]
+    want = O.attention(q[0, L:], k[0, L:], v[0, L:], O.block_causal_allowed(L, L, D))
+    np.testing.assert_allclose(got, want, atol=1e-14)
+
+
+def test_mask_attn_noisy_first_block_sees_only_itself():
+    L, D, Hq, Hkv, d = 32, 8, 2, 1, 4
+    r = np.random.default_rng(10)
+    q, k, v = (r.standard_normal((1, 2 * L, h, d)) for h in (Hq, Hkv, Hkv))
+    got = O.mask_attn(q, k, v, L, D, rows=np.arange(D))[0]
+    want = O.attention(q[0, :D], k[0, :D], v[0, :D])
+    np.testing.assert_allclose(got, want, atol=1e-14)
+
+
+# --------------------------------------------------- token shift (R5)
+def test_token_shift_reads_previous_row():
+    # Row j of the block is the one-hot e_j (scaled), h_prev is e_39, W = I:
+    # the prediction for position p must come out as token p-1 (39 for p=0).
+    H = V = 40
+    h = np.zeros((1, 32, H), np.float32)
+    for j in range(32):
+        h[0, j, j] = 10.0
+    h_prev = np.zeros((1, H), np.float32)
+    h_prev[0, 39] = 10.0
+    W = np.eye(V, H, dtype=np.float32)
+    bits = np.array([0xFFFFFFFF], np.uint32)
+    res = O.confidence_select(h, h_prev, W, bits, 0.0, 32, np.full((1, 32), -1))
+    want = np.array([39] + list(range(31)))
+    np.testing.assert_array_equal(res["argmax"][0], want)
+    p = math.exp(10) / (math.exp(10) + 39)
+    np.testing.assert_allclose(res["pmax"][0], p, rtol=1e-14)
+
+
+def test_shift_only_affects_next_position():
+    r = np.random.default_rng(4)
+    H, V = 16, 64
+    h = r.standard_normal((1, 32, H)).astype(np.float32)
+    hp = r.standard_normal((1, H)).astype(np.float32)
+    W = r.standard_normal((V, H)).astype(np.float32)
+    bits = np.array([0xFFFFFFFF], np.uint32)
+    a = O.confidence_select(h, hp, W, bits, 0.9, 32, np.zeros((1, 32)))
+    h2 = h.copy()
+    h2[0, 10] = 0.0
+    b = O.confidence_select(h2, hp, W, bits, 0.9, 32, np.zeros((1, 32)))
+    diff = np.nonzero(a["pmax"][0] != b["pmax"][0])[0]
+    np.testing.assert_array_equal(diff, [11])
+
+
+# --------------------------------------------- softmax / confidence (R6)
+def test_softmax_stats_hand_case():
+    l = np.log(np.array([[1.0, 2.0, 3.0, 2.0, 1.0]]))
+    st = O.softmax_stats(l)
+    np.testing.assert_allclose(st["pmax"], [1 / 3], rtol=1e-15)
+    assert st["argmax"][0] == 2
+    np.testing.assert_allclose(st["gap"], [math.log(1.5)], rtol=1e-14)
+
+
+def test_softmax_stats_tie_lowest_index():
+    st = O.softmax_stats(np.array([[1.0, 5.0, 5.0, 2.0]]))
+    assert st["argmax"][0] == 1 and st["gap"][0] == 0.0
+
+
+def test_softmax_stats_vs_scipy_and_bounds():
+    l = rng.standard_normal((50, 64)) * 4
+    st = O.softmax_stats(l)
+    ref = np.exp(l.max(1) - scipy.special.logsumexp(l, axis=1))
+    np.testing.assert_allclose(st["pmax"], ref, rtol=1e-13)
+    np.testing.assert_allclose(scipy.special.softmax(l, axis=1).sum(1), 1.0, rtol=1e-14)
+    assert np.all(st["pmax"] <= 1.0) and np.all(st["pmax"] > 1.0 / 64)
+    np.testing.assert_array_equal(st["argmax"], np.argmax(scipy.special.softmax(l, axis=1), 1))
+
+
+def test_lm_logits_bf16_widening_and_slices():
+    W = np.array([[0x3F80, 0xC000], [0x3F00, 0x4040], [0, 0x3E80]], np.uint16)  # [[1,-2],[.5,3],[0,.25]]
+    rows = np.array([[2.0, 1.0]])
+    np.testing.assert_array_equal(O.lm_logits(rows, W, "bf16", cols=2), [[0.0, 4.0, 0.25]])
+
+
+# --------------------------------------------------------- selection (R7)
+def _golden_select_cases():
+    cases = []
+    for ln in open(os.path.join(GOLDEN, "select_cases.txt")):
+        if not ln.strip() or ln.startswith("#"):
+            continue
+        pos, pm, tau, S, want = [f.strip() for f in ln.split(";")]
+        pos = [] if pos == "-" else [int(x) for x in pos.split(",")]
+        pm = [] if pm == "-" else [float(x) for x in pm.split(",")]
+        want = [] if want == "-" else [int(x) for x in want.split(",")]
+        cases.append((pos, pm, float(tau), int(S), want))
+    return cases
+
+
+@pytest.mark.parametrize("case", _golden_select_cases())
+def test_select_golden(case):
+    pos, pm, tau, S, want = case
+    bits = np.array([sum(1 << p for p in pos)], np.uint32)
+    pmax = np.full((1, 32), np.nan)
+    arg = np.full((1, 32), -1)
+    for p, v in zip(pos, pm):
+        pmax[0, p] = v
+        arg[0, p] = 1000 + p
+    tok, un = O.select(pmax, arg, bits, tau, S, np.full((1, 32), -1))
+    assert int(un[0]) == sum(1 << p for p in want)
+    for p in range(32):
+        assert tok[0, p] == (1000 + p if p in want else -1)
+
+
+def _random_pmax(B, seed):
+    r = np.random.default_rng(seed)
+    bits = r.integers(0, 2 ** 32, size=B, dtype=np.uint64).astype(np.uint32)
+    bits[0] = 0
+    bits[1] = 1 << 31
+    return bits, r.random((B, 32)), r.integers(0, 100, size=(B, 32))
+
+
+@pytest.mark.parametrize("S", [1, 2, 4, 8, 16, 32])
+def test_tau_one_unmasks_exactly_one(S):
+    # Threshold 1.0 reduces to standard one-token decoding ([N1] key design 3).
+    bits, pmax, arg = _random_pmax(200, S)
+    pmax[5] = 1.0
+    _, un = O.select(pmax, arg, bits, 1.0, S, np.zeros((200, 32)))
+    for s in range(200):
+        want = 1 if bits[s] else 0
+        assert bin(int(un[s])).count("1") == want
+
+
+@pytest.mark.parametrize("S", [4, 8, 32])
+def test_tau_zero_unmasks_all_candidates_and_subset(S):
+    bits, pmax, arg = _random_pmax(100, 3 + S)
+    pmax = np.maximum(pmax, 1e-9)
+    _, un = O.select(pmax, arg, bits, 0.0, S, np.zeros((100, 32)))
+    for s in range(100):
+        C = O.active_candidates(int(bits[s]), S)
+        assert int(un[s]) == sum(1 << c for c in C)
+    _, un9 = O.select(pmax, arg, bits, 0.9, S, np.zeros((100, 32)))
+    assert np.all((un9 & ~un) == 0)          # unmask subset of candidates
+    assert np.all((un9 & ~bits) == 0)        # only masked positions
+
+
+def test_strict_threshold():
+    pmax = np.full((1, 32), 0.0)
+    pmax[0, :3] = [0.9, 0.9, 0.2]
+    _, un = O.select(pmax, np.zeros((1, 32), int), np.array([0b111], np.uint32), 0.9, 8, np.zeros((1, 32)))
+    assert int(un[0]) == 0b001      # none > tau: fallback to the first of the tied best
+
+
+# ------------------------------------------------------- ambiguity (R8)
+def test_ambiguity_flags():
+    bits = np.array([0b111, 0b11, 0b1], np.uint32)
+    pmax = np.full((3, 32), np.nan)
+    gap = np.full((3, 32), np.nan)
+    pmax[0, :3] = [0.95, 0.90005, 0.1]
+    gap[0, :3] = [1.0, 5e-4, 2.0]
+    pmax[1, :2] = [0.5, 0.50005]
+    gap[1, :2] = [1.0, 1.0]
+    pmax[2, 0] = 0.3
+    gap[2, 0] = 0.3
+    tok, dec = O.ambiguity(pmax, gap, bits, 0.9, 8)
+    np.testing.assert_array_equal(dec, [True, True, False])
+    assert tok[0, 1] and not tok[0, 0] and not tok[1].any()
