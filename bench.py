@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Throughput of one block-diffusion denoising step on B200.
+
+A step is the whole per-step hot path over one batch: bd_block_attn (the
+current 32-token block over its block-level KV cache) followed by
+bd_confidence_select (token shift, LM head, softmax statistics, unmask).
+Metric: masked positions scored per second (every masked position of every
+sequence gets its logits scored once per step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--tau T] [--sub-block S]
+
+Under torchrun every rank runs an independent replica of the workload (the
+batches are independent; no collective on the data path): weak scaling.
+Inputs are synthetic and seeded (no dataset, no trained weights).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from decoding_bd_block_b200 import workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = W.QWEN15B_STEP.name
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+SELECT_KERNEL_SOURCES = ("decoding_bd_block_b200/csrc/select_simt.cu",)
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.STEP_CONFIGS))
+    ap.add_argument("--tau", type=float, default=None)
+    ap.add_argument("--sub-block", type=int, default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    return ap.parse_args(argv)
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; torchrun sets the env)
+# --------------------------------------------------------------------------
+class Dist:
+    def __init__(self, backend: str):
+        import torch.distributed as dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.dist = dist if self.world > 1 else None
+        if self.dist is not None:
+            import datetime
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=180))
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, x: float, device=None) -> float:
+        if self.dist is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, x: float, device=None) -> float:
+        if self.dist is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.lines, self.proc = [], None
+        if gpu_id is None:
+            return
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-i", gpu_id, "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 5:
+            time.sleep(0.02)
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append((time.time(), ln.strip()))
+
+    def mark(self):
+        return time.time()
+
+    def stop(self, t0: float, t1: float):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [ln.split(", ") for t, ln in self.lines if t0 - 0.15 <= t <= t1 + 0.25]
+        rows = [r for r in rows if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's
+    source is unchanged since it was captured (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for src in rec.get("sources", []):
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec.get("source_sha256"):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def source_sha(paths):
+    h = hashlib.sha256()
+    for src in paths:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+# --------------------------------------------------------------------------
+# the oracle as a CPU baseline (test infrastructure, timed as it stands)
+# --------------------------------------------------------------------------
+def oracle_step_sample(cfg, a_in, s_in, frac: float, tau: float, S: int):
+    """One oracle step on a bounded sample: full block attention, and the
+    LM-head statistics / selection over the first `frac` of the vocabulary.
+    Returns the masked-position equivalents scored (frac x masked positions)."""
+    import oracle as O
+    if a_in is not None:
+        for s in range(cfg.batch):
+            c = O.OracleCache(1, cfg.n_heads_kv, cfg.head_dim, cfg.rope_theta)
+            if a_in["prefix_len"][s]:
+                c.commit(0, O.widen(a_in["prefix_k"][s], cfg.dtype),
+                         O.widen(a_in["prefix_v"][s], cfg.dtype))
+            O.block_attn_seq(c.k[0], c.v[0], O.widen(a_in["q"][s], cfg.dtype),
+                             O.widen(a_in["k_blk"][s], cfg.dtype),
+                             O.widen(a_in["v_blk"][s], cfg.dtype), cfg.rope_theta)
+    if s_in is None:
+        return 0.0
+    Vs = max(1, int(round(cfg.vocab * frac)))
+    r = O.confidence_select(s_in["h"], s_in["h_prev"], s_in["W"][:Vs], s_in["masked_bits"], tau, S,
+                            s_in["tokens"], cfg.dtype)
+    return r["n_scored"] * Vs / cfg.vocab
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, a_in, s_in, tau, S, budget_s):
+    """Time the oracle on a sample of the workload for about `budget_s`."""
+    t0 = time.perf_counter()
+    oracle_step_sample(cfg, a_in, s_in, 0.02, tau, S)       # probe: 2% of the vocab
+    probe = max(time.perf_counter() - t0, 1e-3)
+    frac = float(min(1.0, max(0.02, 0.02 * budget_s / probe / 2)))
+    scored, t_total, n = 0.0, 0.0, 0
+    while t_total < budget_s * 0.5 or n == 0:
+        t0 = time.perf_counter()
+        scored += oracle_step_sample(cfg, a_in, s_in, frac, tau, S)
+        t_total += time.perf_counter() - t0
+        n += 1
+    import platform
+    return {"value": scored / t_total, "unit": "masked positions scored/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": (f"{n} oracle step(s) of workload {cfg.name}: full block attention + "
+                       f"LM-head statistics and selection over {frac:.1%} of the vocabulary "
+                       f"({frac:.3f} x {s_in['n_scored'] if s_in else 0} masked positions per step); "
+                       f"fp64 numpy on {platform.processor() or platform.machine()}")}
+
+
+# --------------------------------------------------------------------------
+# arms
+# --------------------------------------------------------------------------
+def run_reference(args, cfg, tau, S):
+    a_in = W.make_attn_inputs(cfg)
+    s_in = W.make_select_inputs(cfg) if cfg.hidden else None
+    if s_in is not None:
+        s_in["n_scored"] = int(sum(bin(int(b)).count("1") for b in s_in["masked_bits"]))
+    t0 = time.perf_counter()
+    oracle_step_sample(cfg, a_in, s_in, 0.02, tau, S)
+    probe = max(time.perf_counter() - t0, 1e-3)
+    per_step_budget = 150.0 / max(1, args.steps + args.warmup)
+    frac = float(min(1.0, max(0.002, 0.02 * per_step_budget / probe)))
+    for _ in range(args.warmup):
+        oracle_step_sample(cfg, a_in, s_in, frac, tau, S)
+    scored, t = 0.0, 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        scored += oracle_step_sample(cfg, a_in, s_in, frac, tau, S)
+        t += time.perf_counter() - t0
+    value = scored / t
+    line = {
+        "metric": "masked positions scored/s per denoise step", "value": value,
+        "unit": "masked positions scored/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "tau": tau, "sub_block": S,
+                   "vocab_fraction_per_step": frac},
+        "cpu_baseline": {"value": value, "unit": "masked positions scored/s", "kind": "oracle",
+                         "cores": blas_threads(),
+                         "sample": f"each step: full block attention + LM-head statistics over "
+                                   f"{frac:.2%} of the vocabulary of workload {cfg.name}"},
+        "e2e": {"value": value, "unit": "masked positions scored/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, cfg, tau, S, dist: Dist):
+    import torch
+
+    from decoding_bd_block_b200 import bd
+    from decoding_bd_block_b200.step import DecodeStep
+
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    a_in = W.make_attn_inputs(cfg)
+    s_in = W.make_select_inputs(cfg) if cfg.hidden else None
+    step = DecodeStep(cfg, a_in, s_in, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step.run(tau, S)
+    torch.cuda.synchronize(dev)
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    launches0 = bd.bd_kernel_launches()
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        if step.attn:
+            step.run_attn()
+        ev[i][1].record(stream)
+        if step.sel:
+            step.run_select(tau, S)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    t_wall1 = time.time()
+    launches = bd.bd_kernel_launches() - launches0
+    clocks = sampler.stop(t_wall0, t_wall1)
+
+    t_attn = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    t_sel = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    t_step = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
+    ms_rank = float(np.mean(t_step))
+    ms = dist.max(ms_rank, dev)
+    n_scored = step.n_scored if step.sel else 0
+    unit_count = n_scored if step.sel else cfg.batch * W.BLOCK * cfg.n_heads_q
+    total_units = dist.sum(float(unit_count), dev)
+    value = total_units / (ms / 1e3)
+
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    if step.sel:
+        w_bytes = cfg.vocab * cfg.hidden * (2 if cfg.dtype == "bf16" else 4)
+        rows_bytes = n_scored * cfg.hidden * (2 if cfg.dtype == "bf16" else 4)
+        alg = w_bytes + rows_bytes
+        t_dom = float(np.mean(t_sel)) / 1e3
+        traffic = recorded_traffic("lmhead")
+        roofline = {"kernel": "bd_confidence_select (LM-head vocab stream; whole call timed)",
+                    "bound": "hbm", "achieved": alg / t_dom / 1e9, "peak": hbm, "unit": "GB/s",
+                    "frac": alg / t_dom / 1e9 / hbm, "traffic": traffic,
+                    "algorithmic_bytes_per_launch": alg, "peak_source": peak_kind}
+    else:
+        roofline = None
+
+    e2e = None
+    if not args.no_e2e and step.sel:
+        e2e = measure_e2e(step, cfg, tau, S, flush, dev, dist, max(10, K // 4))
+
+    line = {
+        "metric": "masked positions scored/s per denoise step",
+        "value": value, "unit": "masked positions scored/s", "n_gpus": dist.world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "n_heads_q": cfg.n_heads_q,
+                   "n_heads_kv": cfg.n_heads_kv, "head_dim": cfg.head_dim,
+                   "prefix_tokens": [int(x) for x in a_in["prefix_len"]],
+                   "hidden": cfg.hidden, "vocab": cfg.vocab, "tau": tau, "sub_block": S,
+                   "masked_positions_per_step": n_scored,
+                   "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
+                   "parallelism": f"replicas x{dist.world} (independent batches)"},
+        "breakdown_ms": {"bd_block_attn": float(np.mean(t_attn)),
+                         "bd_confidence_select": float(np.mean(t_sel))},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "timed_region_wall_s": t_wall1 - t_wall0,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        if s_in is not None:
+            s_in["n_scored"] = n_scored
+        line["cpu_baseline"] = cpu_baseline(cfg, a_in, s_in, tau, S, args.cpu_budget_s)
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def measure_e2e(step, cfg, tau, S, flush, dev, dist, K):
+    """Same metric through the public API with the step's inputs on pinned host
+    memory: H2D of the step inputs and D2H of tokens + unmask bits are inside
+    the timed region of every step."""
+    import torch
+    host_in = []
+    for name in ("q", "k_blk", "v_blk", "h", "h_prev", "masked", "tokens_in"):
+        t = getattr(step, name, None)
+        if t is not None:
+            host_in.append((t, t.cpu().pin_memory()))
+    tok_h = torch.empty(step.tokens.shape, dtype=step.tokens.dtype).pin_memory()
+    un_h = torch.empty(step.unmask.shape, dtype=step.unmask.dtype).pin_memory()
+    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
+    d2h = tok_h.numel() * tok_h.element_size() + un_h.numel() * un_h.element_size()
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    dist.barrier()
+    for _ in range(K):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for dst, src in host_in:
+            dst.copy_(src, non_blocking=True)
+        step.tokens.copy_(step.tokens_in)
+        step.run(tau, S)
+        tok_h.copy_(step.tokens, non_blocking=True)
+        un_h.copy_(step.unmask, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = dist.max(float(np.mean(times)), dev)
+    total = dist.sum(float(step.n_scored), dev)
+    return {"value": total / (ms / 1e3), "unit": "masked positions scored/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    cfg = W.STEP_CONFIGS[args.workload]
+    tau = args.tau if args.tau is not None else cfg.taus[0]
+    S = args.sub_block if args.sub_block is not None else cfg.sub_block
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if world > 1 and rank != 0:
+            return 0
+        run_reference(args, cfg, tau, S)
+        return 0
+    dist = Dist("nccl")
+    try:
+        run_ours(args, cfg, tau, S, dist)
+    finally:
+        dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,135 @@
+// Shared device helpers of libbd (element access, RoPE angles, fast exp2,
+// warp reductions) and the internal launcher interface used by bd_api.cu.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/bd.h"
+
+namespace bd {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int kBlock = BD_BLOCK;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------- elements
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(bf16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ bf16 from_f32<bf16>(float x) { return __float2bfloat16_rn(x); }
+
+// 2^x on the MUFU unit (hardware approximation, relative error ~2^-22).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// --------------------------------------------------------------- warp ops
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ------------------------------------------------------------------ RoPE
+// cos/sin of pos * theta^(-2j/d), evaluated in double precision so that the
+// angle stays exact to ~1e-12 rad at positions in the tens of thousands.
+__device__ __forceinline__ void rope_cos_sin(long long pos, double inv_freq, float* c, float* s) {
+  double sd, cd;
+  sincos(static_cast<double>(pos) * inv_freq, &sd, &cd);
+  *c = static_cast<float>(cd);
+  *s = static_cast<float>(sd);
+}
+
+__device__ __forceinline__ double rope_inv_freq(int j, int d, double theta) {
+  return pow(theta, -2.0 * static_cast<double>(j) / static_cast<double>(d));
+}
+
+// ------------------------------------------------- (max, sum, argmax) triple
+// Running softmax statistics of a set of logits: m = max, s = sum exp(l - m),
+// a = lowest index attaining m.  combine() is associative and commutative.
+struct Stat {
+  float m;
+  float s;
+  int a;
+};
+__device__ __forceinline__ Stat stat_empty() { return Stat{-INFINITY, 0.f, 0x7fffffff}; }
+__device__ __forceinline__ Stat stat_combine(Stat x, Stat y) {
+  if (y.m == -INFINITY) return x;
+  if (x.m == -INFINITY) return y;
+  Stat r;
+  r.m = fmaxf(x.m, y.m);
+  r.s = x.s * expf(x.m - r.m) + y.s * expf(y.m - r.m);
+  if (x.m == y.m) r.a = min(x.a, y.a);
+  else r.a = (x.m > y.m) ? x.a : y.a;
+  return r;
+}
+
+// Process-wide count of kernels enqueued by the library (bd_kernel_launches).
+void count_launches(int n);
+
+__host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace bd
+
+// ---------------------------------------------------------------------------
+// Internal launchers (defined in the kernel files, called by bd_api.cu).
+// Arguments are validated by the caller; each returns cudaGetLastError().
+// ---------------------------------------------------------------------------
+namespace bd {
+
+struct CommitArgs {
+  int n_seqs;
+  int n_new_blocks;
+  int seq_ids[256];
+  int first_block[256];  // n_blocks_host[s] before the commit
+};
+
+cudaError_t launch_cache_commit(const bd_attn_shape& sh, const bd_kv_cache& c, const void* k,
+                                const void* v, const CommitArgs& a, cudaStream_t st);
+
+// Block attention plan: pages per split-KV chunk and the largest chunk count.
+struct AttnPlan {
+  int pages_per_chunk;
+  int max_chunks;
+  size_t off_q, off_blk, off_o, off_ml, total;
+};
+AttnPlan plan_block_attn(const bd_attn_shape& sh, const bd_kv_cache& c);
+cudaError_t launch_block_attn(const bd_attn_shape& sh, const bd_kv_cache& c, const AttnPlan& p,
+                              const void* q, const void* k, const void* v, void* out, void* ws,
+                              cudaStream_t st);
+
+struct SelectPlan {
+  int n_split;       // vocab splits (partials per row)
+  int rows_alloc;    // packed-row capacity (>= 32 * batch, padded)
+  size_t off_rows, off_rowmap, off_posrow, off_count, off_pm, off_ps, off_pa, total;
+};
+SelectPlan plan_confidence_select(int dtype, int batch, int hidden, int vocab);
+cudaError_t launch_confidence_select(int dtype, int batch, int hidden, int vocab,
+                                     const SelectPlan& p, const void* h, const void* h_prev,
+                                     const void* w, const uint32_t* masked, float tau,
+                                     int sub_block, int32_t* tokens, uint32_t* unmask,
+                                     float* pmax_out, int32_t* argmax_out, void* ws,
+                                     cudaStream_t st);
+
+cudaError_t launch_block_mask_attn(const bd_attn_shape& sh, const void* q, const void* k,
+                                   const void* v, void* out, int n_seqs, int L, int block,
+                                   cudaStream_t st);
+
+}  // namespace bd

@@ -1,0 +1,252 @@
+// bd_confidence_select: token shift -> LM head -> (max, sum, argmax) per row
+// -> confidence-aware unmask ("Fast-dLLM v2: Efficient Block-Diffusion LLM",
+// key designs 2-4; Fast-dLLM v1 article, confidence-aware parallel decoding).
+//
+// Launches:
+//   1. gather_rows     packs, per masked position i, hidden row i-1 (h_prev
+//                      for i = 0) into a dense [M][H] matrix; records the
+//                      row of each position and M;
+//   2. lm head stats   vocab-split: each CTA folds its vocab range into a
+//                      running (max, sum exp, argmax) per row; logits stay on
+//                      chip (CUDA-core tile here, tcgen05 in select_tc.cu);
+//   3. merge_select    merges the partials of every row, turns them into
+//                      p_max and the token, and applies the unmask rule.
+#include "bd_common.cuh"
+
+namespace bd {
+
+// grid (batch), 256 threads.
+template <typename T>
+__global__ void __launch_bounds__(256) gather_rows_kernel(
+    const T* __restrict__ h, const T* __restrict__ h_prev, const uint32_t* __restrict__ masked,
+    int B, int H, T* __restrict__ rows, int32_t* __restrict__ rowmap,
+    int32_t* __restrict__ posrow, int32_t* __restrict__ count, int rows_alloc) {
+  __shared__ int red[8];
+  const int s = blockIdx.x;
+  int acc = 0;
+  for (int x = threadIdx.x; x < s; x += blockDim.x) acc += __popc(masked[x]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = acc;
+  __syncthreads();
+  int off = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) off += red[w];
+  const uint32_t bits = masked[s];
+  if (threadIdx.x < kBlock) {
+    const int i = threadIdx.x;
+    int r = -1;
+    if ((bits >> i) & 1u) {
+      r = off + __popc(bits & ((1u << i) - 1u));
+      rowmap[r] = s * kBlock + i;
+    }
+    posrow[s * kBlock + i] = r;
+  }
+  int k = 0;
+  for (int i = 0; i < kBlock; ++i) {
+    if (!((bits >> i) & 1u)) continue;
+    const T* src = (i == 0) ? h_prev + static_cast<size_t>(s) * H
+                            : h + (static_cast<size_t>(s) * kBlock + i - 1) * H;
+    T* dst = rows + static_cast<size_t>(off + k) * H;
+    for (int x = threadIdx.x; x < H; x += blockDim.x) dst[x] = src[x];
+    ++k;
+  }
+  if (s == B - 1) {
+    const int total = off + __popc(bits);
+    if (threadIdx.x == 0) *count = total;
+    const int pad_end = min(rows_alloc, (total + 15) / 16 * 16);
+    for (size_t x = static_cast<size_t>(total) * H + threadIdx.x;
+         x < static_cast<size_t>(pad_end) * H; x += blockDim.x)
+      rows[x] = from_f32<T>(0.f);
+  }
+}
+
+// grid (n_split, rows_alloc / 32), 256 threads.  Tile: 64 vocab x 32 rows,
+// K-steps of 32; CTA x strides over vocab tiles x, x + n_split, ...
+template <typename T>
+__global__ void __launch_bounds__(256) lmhead_simt_kernel(
+    const T* __restrict__ rows, const T* __restrict__ w, const int32_t* __restrict__ count,
+    int H, int V, int n_split, int rows_alloc, float* __restrict__ pm, float* __restrict__ ps,
+    int32_t* __restrict__ pa) {
+  __shared__ float Ws[32][68];
+  __shared__ float Rs[32][36];
+  __shared__ float Ls[32][65];
+  const int M = *count;
+  const int r0 = blockIdx.y * 32;
+  if (r0 >= M) return;
+  const int tid = threadIdx.x;
+  const int tv = tid % 16, tr = tid / 16;
+  float run_m = -INFINITY, run_s = 0.f;
+  int run_a = 0x7fffffff;
+  for (int vt = blockIdx.x; vt * 64 < V; vt += n_split) {
+    const int v0 = vt * 64;
+    float acc[2][4] = {};
+    for (int k0 = 0; k0 < H; k0 += 32) {
+      __syncthreads();
+      for (int i = tid; i < 64 * 32; i += 256) {
+        const int vv = i / 32, kk = i % 32;
+        const int vg = v0 + vv, kg = k0 + kk;
+        Ws[kk][vv] = (vg < V && kg < H) ? to_f32(w[static_cast<size_t>(vg) * H + kg]) : 0.f;
+      }
+      for (int i = tid; i < 32 * 32; i += 256) {
+        const int rr = i / 32, kk = i % 32;
+        const int rg = r0 + rr, kg = k0 + kk;
+        Rs[kk][rr] = (rg < M && kg < H) ? to_f32(rows[static_cast<size_t>(rg) * H + kg]) : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int kk = 0; kk < 32; ++kk) {
+        float wv[4], rv[2];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) wv[b] = Ws[kk][tv * 4 + b];
+#pragma unroll
+        for (int a = 0; a < 2; ++a) rv[a] = Rs[kk][tr * 2 + a];
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(rv[a], wv[b], acc[a][b]);
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) Ls[tr * 2 + a][tv * 4 + b] = acc[a][b];
+    __syncthreads();
+    if (tid < 32) {
+      for (int vv = 0; vv < 64 && v0 + vv < V; ++vv) {
+        const float x = Ls[tid][vv];
+        if (x > run_m) {
+          run_s = run_s * expf(run_m - x) + 1.f;
+          run_m = x;
+          run_a = v0 + vv;
+        } else {
+          run_s += expf(x - run_m);
+        }
+      }
+    }
+  }
+  if (tid < 32 && r0 + tid < M) {
+    const size_t idx = static_cast<size_t>(blockIdx.x) * rows_alloc + r0 + tid;
+    pm[idx] = run_m;
+    ps[idx] = run_s;
+    pa[idx] = run_a;
+  }
+}
+
+// grid (batch), 32 threads: thread i owns position i of sequence s.
+__global__ void __launch_bounds__(32) merge_select_kernel(
+    const int32_t* __restrict__ posrow, const uint32_t* __restrict__ masked, int n_split,
+    int rows_alloc, const float* __restrict__ pm, const float* __restrict__ ps,
+    const int32_t* __restrict__ pa, float tau, int S, int32_t* __restrict__ tokens,
+    uint32_t* __restrict__ unmask, float* __restrict__ pmax_out, int32_t* __restrict__ argmax_out) {
+  const int s = blockIdx.x, i = threadIdx.x;
+  const uint32_t bits = masked[s];
+  const bool is_m = (bits >> i) & 1u;
+  float p = 0.f;
+  int tok = -1;
+  if (is_m) {
+    const int r = posrow[s * kBlock + i];
+    Stat st = stat_empty();
+    for (int k = 0; k < n_split; ++k) {
+      const size_t idx = static_cast<size_t>(k) * rows_alloc + r;
+      st = stat_combine(st, Stat{pm[idx], ps[idx], pa[idx]});
+    }
+    p = 1.f / st.s;
+    tok = st.a;
+  }
+  // Candidates: masked positions of the lowest sub-block that has one.
+  const int first = bits ? __ffs(static_cast<int>(bits)) - 1 : 0;
+  const int k0 = (first / S) * S;
+  const bool cand = is_m && i >= k0 && i < k0 + S;
+  const uint32_t above = __ballot_sync(0xffffffffu, cand && p > tau);
+  uint32_t U = above;
+  if (!above) {
+    float bp = cand ? p : -1.f;
+    int bi = cand ? i : 32;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float op = __shfl_xor_sync(0xffffffffu, bp, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (op > bp || (op == bp && oi < bi)) {
+        bp = op;
+        bi = oi;
+      }
+    }
+    U = (bi < 32) ? (1u << bi) : 0u;
+  }
+  if ((U >> i) & 1u) tokens[s * kBlock + i] = tok;
+  if (i == 0) unmask[s] = U;
+  if (pmax_out) pmax_out[s * kBlock + i] = is_m ? p : __int_as_float(0x7fc00000);
+  if (argmax_out) argmax_out[s * kBlock + i] = is_m ? tok : -1;
+}
+
+// -------------------------------------------------------------- host side
+SelectPlan plan_confidence_select(int dtype, int batch, int hidden, int vocab) {
+  SelectPlan p{};
+  p.rows_alloc = static_cast<int>(align_up(static_cast<size_t>(batch) * kBlock, 256));
+  const int vtiles = (vocab + 63) / 64;
+  const int rtiles = p.rows_alloc / 32;
+  int ns = (4 * 148 + rtiles - 1) / rtiles;
+  if (ns > vtiles) ns = vtiles;
+  if (ns < 1) ns = 1;
+  p.n_split = ns;
+  const size_t es = dtype == BD_BF16 ? 2 : 4;
+  size_t off = 0;
+  p.off_rows = off;
+  off = align_up(off + static_cast<size_t>(p.rows_alloc) * hidden * es, 256);
+  p.off_rowmap = off;
+  off = align_up(off + static_cast<size_t>(p.rows_alloc) * 4, 256);
+  p.off_posrow = off;
+  off = align_up(off + static_cast<size_t>(batch) * kBlock * 4, 256);
+  p.off_count = off;
+  off = align_up(off + 4, 256);
+  const size_t part = static_cast<size_t>(p.n_split) * p.rows_alloc * 4;
+  p.off_pm = off;
+  off = align_up(off + part, 256);
+  p.off_ps = off;
+  off = align_up(off + part, 256);
+  p.off_pa = off;
+  off = align_up(off + part, 256);
+  p.total = off;
+  return p;
+}
+
+template <typename T>
+static cudaError_t launch_select_t(int batch, int hidden, int vocab, const SelectPlan& p,
+                                   const void* h, const void* h_prev, const void* w,
+                                   const uint32_t* masked, float tau, int S, int32_t* tokens,
+                                   uint32_t* unmask, float* pmax_out, int32_t* argmax_out,
+                                   void* ws, cudaStream_t st) {
+  char* base = static_cast<char*>(ws);
+  T* rows = reinterpret_cast<T*>(base + p.off_rows);
+  int32_t* rowmap = reinterpret_cast<int32_t*>(base + p.off_rowmap);
+  int32_t* posrow = reinterpret_cast<int32_t*>(base + p.off_posrow);
+  int32_t* count = reinterpret_cast<int32_t*>(base + p.off_count);
+  float* pm = reinterpret_cast<float*>(base + p.off_pm);
+  float* ps = reinterpret_cast<float*>(base + p.off_ps);
+  int32_t* pa = reinterpret_cast<int32_t*>(base + p.off_pa);
+  gather_rows_kernel<T><<<batch, 256, 0, st>>>(static_cast<const T*>(h),
+                                               static_cast<const T*>(h_prev), masked, batch,
+                                               hidden, rows, rowmap, posrow, count, p.rows_alloc);
+  lmhead_simt_kernel<T><<<dim3(p.n_split, p.rows_alloc / 32), 256, 0, st>>>(
+      rows, static_cast<const T*>(w), count, hidden, vocab, p.n_split, p.rows_alloc, pm, ps, pa);
+  merge_select_kernel<<<batch, 32, 0, st>>>(posrow, masked, p.n_split, p.rows_alloc, pm, ps, pa,
+                                            tau, S, tokens, unmask, pmax_out, argmax_out);
+  count_launches(3);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_confidence_select(int dtype, int batch, int hidden, int vocab,
+                                     const SelectPlan& p, const void* h, const void* h_prev,
+                                     const void* w, const uint32_t* masked, float tau,
+                                     int sub_block, int32_t* tokens, uint32_t* unmask,
+                                     float* pmax_out, int32_t* argmax_out, void* ws,
+                                     cudaStream_t st) {
+  if (dtype == BD_BF16)
+    return launch_select_t<bf16>(batch, hidden, vocab, p, h, h_prev, w, masked, tau, sub_block,
+                                 tokens, unmask, pmax_out, argmax_out, ws, st);
+  return launch_select_t<float>(batch, hidden, vocab, p, h, h_prev, w, masked, tau, sub_block,
+                                tokens, unmask, pmax_out, argmax_out, ws, st);
+}
+
+}  // namespace bd

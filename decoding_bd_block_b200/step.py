@@ -1,0 +1,98 @@
+"""Device-side set-up of one decoding step, driven through the C ABI.
+
+A thin host harness: it allocates the caller-owned buffers with torch (the
+KV cache, inputs, outputs and workspaces), fills the block-level cache with
+``bd_cache_commit`` and runs the step as ``bd_block_attn`` followed by
+``bd_confidence_select``.  All arithmetic happens in libbd's kernels.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import bd
+from .workloads import BLOCK, StepConfig
+
+
+def to_device(a: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
+    """Upload fp32 data, or bf16 bit patterns (uint16) as a bfloat16 tensor."""
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+
+def torch_dtype(dtype: str):
+    return torch.bfloat16 if dtype == "bf16" else torch.float32
+
+
+class BlockCacheState:
+    """KV cache of a batch, filled with the pre-RoPE prefix K/V of a workload."""
+
+    def __init__(self, cfg: StepConfig, prefix_len, prefix_k=None, prefix_v=None,
+                 extra_blocks: int = 2, device="cuda", page_table=None, n_pages=None):
+        self.cfg = cfg
+        self.shape = bd.make_shape(cfg.n_heads_q, cfg.n_heads_kv, cfg.head_dim, cfg.dtype,
+                                   cfg.rope_theta)
+        P = np.asarray(prefix_len)
+        self.max_blocks = int(P.max()) // BLOCK + extra_blocks
+        self.cache = bd.KVCache(self.shape, cfg.batch, self.max_blocks, device,
+                                n_pages=n_pages, page_table=page_table)
+        if prefix_k is not None:
+            for s in range(cfg.batch):
+                nb = int(P[s]) // BLOCK
+                if nb == 0:
+                    continue
+                k = to_device(prefix_k[s], cfg.dtype, device)
+                v = to_device(prefix_v[s], cfg.dtype, device)
+                bd.bd_cache_commit(self.cache, k, v, [s], nb)
+
+
+class DecodeStep:
+    """Buffers of one denoising step: block attention + confidence select."""
+
+    def __init__(self, cfg: StepConfig, attn_in: dict | None, sel_in: dict | None,
+                 device="cuda", cache: BlockCacheState | None = None):
+        self.cfg = cfg
+        B, dt = cfg.batch, cfg.dtype
+        self.attn = attn_in is not None
+        self.sel = sel_in is not None
+        if self.attn:
+            self.cstate = cache or BlockCacheState(cfg, attn_in["prefix_len"], attn_in["prefix_k"],
+                                                   attn_in["prefix_v"], device=device)
+            self.q = to_device(attn_in["q"], dt, device)
+            self.k_blk = to_device(attn_in["k_blk"], dt, device)
+            self.v_blk = to_device(attn_in["v_blk"], dt, device)
+            self.out = torch.empty_like(self.q)
+            n = bd.bd_block_attn_workspace_size(self.cstate.cache)
+            self.attn_ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+        if self.sel:
+            self.W = to_device(sel_in["W"], dt, device)
+            self.h = to_device(sel_in["h"], dt, device)
+            self.h_prev = to_device(sel_in["h_prev"], dt, device)
+            self.masked_host = np.ascontiguousarray(sel_in["masked_bits"], dtype=np.uint32)
+            self.masked = torch.from_numpy(self.masked_host.view(np.int32)).to(device)
+            self.tokens_in = torch.from_numpy(np.ascontiguousarray(sel_in["tokens"], np.int32)).to(device)
+            self.tokens = self.tokens_in.clone()
+            self.unmask = torch.zeros(B, dtype=torch.int32, device=device)
+            self.pmax = torch.empty((B, BLOCK), dtype=torch.float32, device=device)
+            self.argmax = torch.empty((B, BLOCK), dtype=torch.int32, device=device)
+            n = bd.bd_confidence_select_workspace_size(dt, B, cfg.hidden, cfg.vocab)
+            self.sel_ws = torch.empty(n, dtype=torch.uint8, device=device)
+            self.n_scored = int(sum(bin(int(b)).count("1") for b in self.masked_host))
+
+    def run_attn(self, stream=None):
+        bd.bd_block_attn(self.cstate.cache, self.q, self.k_blk, self.v_blk, self.out,
+                         self.attn_ws, stream=stream)
+
+    def run_select(self, tau: float, sub_block: int, stream=None, outputs=True):
+        cfg = self.cfg
+        bd.bd_confidence_select(cfg.dtype, cfg.batch, cfg.hidden, cfg.vocab, self.h, self.h_prev,
+                                self.W, self.masked, tau, sub_block, self.tokens, self.unmask,
+                                self.pmax if outputs else None, self.argmax if outputs else None,
+                                self.sel_ws, stream=stream)
+
+    def run(self, tau: float, sub_block: int, stream=None):
+        if self.attn:
+            self.run_attn(stream)
+        if self.sel:
+            self.run_select(tau, sub_block, stream)

@@ -1,0 +1,202 @@
+/*
+ * bd.h -- C ABI of libbd: one denoising step of block-diffusion decoding
+ * (Fast-dLLM v2) on an NVIDIA B200 (sm_100a).
+ *
+ * Method sources, cited by page title and section:
+ *   [N1] "Fast-dLLM v2: Efficient Block-Diffusion LLM", paper notes
+ *        (papernotes.org), "Overall framework" and "Key designs" 1-4.
+ *   [N2] Fast-dLLM (v1) article (senqingzn.com), "Core techniques" item 2,
+ *        confidence-aware parallel decoding.
+ *   [N4] "Fast-dLLM v2: 2.5x inference speedup" (aigc.bar), "Acceleration
+ *        engine" items 1 (hierarchical cache) and 2 (parallel decoding).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - A block is BD_BLOCK = 32 tokens.  Tensors are dense, row-major, in the
+ *   element type named by a bd_dtype (fp32, or bf16 with fp32 arithmetic).
+ * - Pointers marked "device" must be CUDA device memory of the current
+ *   device; "host" pointers are read on the host during the call only.
+ * - The library allocates nothing and keeps no state between calls: the
+ *   caller owns every buffer, the KV cache and the scratch workspace.  Ask
+ *   for the workspace size with the matching *_workspace_size call.
+ * - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream) and the call returns without synchronising.
+ * - Every entry point returns a bd_status.  Argument errors are found on the
+ *   host before anything is launched (nothing is enqueued then).  BD_ERR_CUDA
+ *   reports a launch failure; the CUDA error string is then available from
+ *   bd_last_cuda_error_string().  Nothing throws across this boundary.
+ * - Calls on the same stream are ordered; calls that share a workspace or a
+ *   cache must not run concurrently on different streams.
+ */
+#ifndef BD_H_
+#define BD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BD_BLOCK 32
+
+#if defined(__GNUC__)
+#define BD_API __attribute__((visibility("default")))
+#else
+#define BD_API
+#endif
+
+typedef enum {
+  BD_OK = 0,
+  BD_ERR_INVALID_ARG = -1, /* null pointer, bad size or shape            */
+  BD_ERR_UNSUPPORTED = -2, /* shape or dtype this build does not handle  */
+  BD_ERR_CAPACITY = -3,    /* KV cache page table / pages exhausted      */
+  BD_ERR_WORKSPACE = -4,   /* workspace missing or too small             */
+  BD_ERR_CUDA = -5         /* a CUDA launch or runtime call failed       */
+} bd_status;
+
+typedef enum { BD_F32 = 0, BD_BF16 = 1 } bd_dtype;
+
+/* Attention geometry.  Query head h reads KV head h / (n_heads_q /
+ * n_heads_kv) (contiguous groups).  head_dim is 64 or 128.  rope_theta is
+ * the RoPE base: pair (j, j + d/2) rotates by pos * rope_theta^(-2j/d). */
+typedef struct {
+  int32_t n_heads_q;
+  int32_t n_heads_kv;
+  int32_t head_dim;
+  int32_t dtype;     /* bd_dtype of q, k, v, cache pages and outputs */
+  double rope_theta;
+} bd_attn_shape;
+
+/* Block-level KV cache ([N1] key design 3; [N4] item 1): per sequence, the
+ * K and V of every finished block, each block stored as one page.  Keys are
+ * stored already rotated (RoPE at their absolute positions).
+ *
+ *   pages       device, [n_pages][2][n_heads_kv][32][head_dim] of dtype;
+ *               index 0 of the second axis is K, 1 is V.
+ *   page_table  device, [batch][max_blocks] int32: physical page of logical
+ *               block b of sequence s (caller-assigned, distinct pages).
+ *   n_blocks    device, [batch] int32: finished blocks per sequence.
+ *   *_host      host mirrors of page_table and n_blocks with the same
+ *               contents; the library reads them for validation and launch
+ *               sizing and keeps n_blocks_host in step on commit.
+ */
+typedef struct {
+  void* pages;
+  int64_t n_pages;
+  int32_t* page_table;
+  const int32_t* page_table_host;
+  int32_t* n_blocks;
+  int32_t* n_blocks_host;
+  int32_t batch;
+  int32_t max_blocks;
+} bd_kv_cache;
+
+/* bd_cache_commit -- append finished blocks to the block-level KV cache.
+ *
+ * [N1] key design 3 / [N4] item 1: once a block is fully decoded its K/V are
+ * kept as read-only context for every later block, exactly like an
+ * autoregressive KV cache.
+ *
+ *   k, v      device, [n_seqs][32 * n_new_blocks][n_heads_kv][head_dim]
+ *             (k before RoPE).
+ *   seq_ids   host, [n_seqs] distinct sequence indices in [0, batch).
+ * For each listed sequence s with P = 32 * n_blocks_host[s], token t of the
+ * input is written, k rotated at absolute position P + t, into page
+ * page_table[s][n_blocks_host[s] + t / 32], row t % 32; then n_blocks (device
+ * and host) grows by n_new_blocks.  Errors: BD_ERR_CAPACITY when
+ * n_blocks_host[s] + n_new_blocks > max_blocks; BD_ERR_INVALID_ARG for a
+ * page id outside [0, n_pages) or a repeated / out-of-range sequence. */
+BD_API int bd_cache_commit(const bd_attn_shape* shape, bd_kv_cache* cache,
+                    const void* k, const void* v, const int32_t* seq_ids,
+                    int32_t n_seqs, int32_t n_new_blocks, void* stream);
+
+/* bd_block_attn -- attention of the current block over the cache.
+ *
+ * [N1] overall framework and key design 3; [N4] "block-internal parallel,
+ * block-causal": every query of the current 32-token block sees all cached
+ * keys of its sequence and all 32 keys of its own block, unmasked.
+ *
+ *   q      device, [batch][32][n_heads_q][head_dim], before RoPE
+ *   k_blk  device, [batch][32][n_heads_kv][head_dim], before RoPE
+ *   v_blk  device, [batch][32][n_heads_kv][head_dim]
+ *   out    device, [batch][32][n_heads_q][head_dim], written
+ * q and k_blk are rotated at positions P..P+31 (P = 32 * n_blocks[s]);
+ * out = softmax(q K^T / sqrt(head_dim)) V over [cached keys ; block keys].
+ * batch is cache->batch.  Workspace: bd_block_attn_workspace_size() bytes,
+ * 256-byte aligned; its size depends on n_blocks_host, so ask again after
+ * the cache grows. */
+BD_API int bd_block_attn_workspace_size(const bd_attn_shape* shape,
+                                 const bd_kv_cache* cache, size_t* bytes);
+BD_API int bd_block_attn(const bd_attn_shape* shape, const bd_kv_cache* cache,
+                  const void* q, const void* k_blk, const void* v_blk,
+                  void* out, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/* bd_confidence_select -- confidence-aware parallel unmask of one step.
+ *
+ * [N1] key designs 2-4, [N2] item 2, [N4] item 2.  For every masked
+ * position i of each sequence (bit i of masked_bits[s]):
+ *   row    = hidden row i-1 of the block, or h_prev[s] for i = 0 (token
+ *            shift, key design 2);
+ *   l      = row . w_lm[v] for every vocab entry v (logits never stored);
+ *   token  = argmax_v l (lowest v on ties); p_max = 1 / sum_v exp(l - max l).
+ * Candidates are the masked positions of the lowest sub-block of
+ * `sub_block` positions that still holds a masked position (key design 4).
+ * Every candidate with p_max > tau is unmasked; if there is none, the single
+ * candidate with the largest p_max is (lowest position on ties).
+ *
+ *   dtype        element type of h, h_prev and w_lm
+ *   h            device, [batch][32][hidden]
+ *   h_prev       device, [batch][hidden]
+ *   w_lm         device, [vocab][hidden]
+ *   masked_bits  device, [batch] uint32; not modified
+ *   tokens       device, [batch][32] int32; unmasked positions receive
+ *                their token, all others are left as they are
+ *   unmask_bits  device, [batch] uint32 out: positions unmasked this step
+ *   pmax_out     device, [batch][32] float or NULL: p_max per masked
+ *                position, NaN elsewhere
+ *   argmax_out   device, [batch][32] int32 or NULL: token per masked
+ *                position, -1 elsewhere
+ * sub_block must divide 32; 0 <= tau.  Workspace: see
+ * bd_confidence_select_workspace_size(). */
+BD_API int bd_confidence_select_workspace_size(int32_t dtype, int32_t batch,
+                                        int32_t hidden, int32_t vocab,
+                                        size_t* bytes);
+BD_API int bd_confidence_select(int32_t dtype, int32_t batch, int32_t hidden,
+                         int32_t vocab, const void* h, const void* h_prev,
+                         const void* w_lm, const uint32_t* masked_bits,
+                         float tau, int32_t sub_block, int32_t* tokens,
+                         uint32_t* unmask_bits, float* pmax_out,
+                         int32_t* argmax_out, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* bd_block_mask_attn -- attention of the training forward under the 2L x 2L
+ * complementary mask ([N1] key design 2).
+ *
+ * Each of the n_seqs entries (one per sample and mask view) is the noisy
+ * stream x_t (rows 0..L-1) followed by the clean stream x_0 (rows L..2L-1).
+ * With blk(i) = (i mod L) / block: a noisy query sees the noisy keys of its
+ * own block and the clean keys of earlier blocks; a clean query sees the
+ * clean keys of its own and earlier blocks; no clean query sees a noisy key.
+ *
+ *   q     device, [n_seqs][2L][n_heads_q][head_dim] (already rotated)
+ *   k, v  device, [n_seqs][2L][n_heads_kv][head_dim]
+ *   out   device, [n_seqs][2L][n_heads_q][head_dim], written
+ * block must divide L; shape->rope_theta is ignored. */
+BD_API int bd_block_mask_attn(const bd_attn_shape* shape, const void* q,
+                       const void* k, const void* v, void* out,
+                       int32_t n_seqs, int32_t L, int32_t block, void* stream);
+
+/* Human-readable name of a bd_status value. */
+BD_API const char* bd_status_string(int status);
+/* Text of the last CUDA error seen by a call of this thread (or ""). */
+BD_API const char* bd_last_cuda_error_string(void);
+/* Number of CUDA kernels this library has enqueued in this process so far
+ * (all threads).  A diagnostic for measuring launches per step. */
+BD_API long long bd_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BD_H_ */

@@ -1,0 +1,259 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Same seeded inputs on both sides.  Unmask decisions and tokens must be
+bit-exact outside the ambiguity flags; attention within max-abs 1e-5 (fp32
+storage) or 2e-2 (bf16 storage); p_max within 1e-4.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import oracle as O
+from decoding_bd_block_b200 import workloads as W
+from parity_util import ATOL, compare_select, oracle_block_attn
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from decoding_bd_block_b200 import bd  # noqa: F401  (fails loudly if libbd.so is missing)
+    torch.cuda.init()
+
+
+def _step(cfg, attn=True, sel=True, prefix=None):
+    from decoding_bd_block_b200.step import DecodeStep
+    a = W.make_attn_inputs(cfg, prefix) if attn else None
+    s = W.make_select_inputs(cfg) if sel else None
+    return a, s, DecodeStep(cfg, a, s)
+
+
+# ------------------------------------------------------------ cache commit
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_commit_pages_match_oracle(dtype):
+    from decoding_bd_block_b200.step import BlockCacheState
+    cfg = dataclasses.replace(W.TINY_F32, dtype=dtype, batch=3, rope_theta=1e6, seed=77)
+    P = np.array([96, 0, 320])
+    a = W.make_attn_inputs(cfg, P)
+    st = BlockCacheState(cfg, P, a["prefix_k"], a["prefix_v"])
+    torch.cuda.synchronize()
+    pages = st.cache.pages.float().cpu().numpy()
+    pt = st.cache.page_table_host
+    assert list(st.cache.n_blocks_host) == [3, 0, 10]
+    assert st.cache.n_blocks.cpu().tolist() == [3, 0, 10]
+    for s in (0, 2):
+        c = O.OracleCache(1, cfg.n_heads_kv, cfg.head_dim, cfg.rope_theta)
+        c.commit(0, O.widen(a["prefix_k"][s], dtype), O.widen(a["prefix_v"][s], dtype))
+        for b in range(P[s] // 32):
+            k_gpu = pages[pt[s, b], 0].transpose(1, 0, 2)   # [32, Hkv, d]
+            v_gpu = pages[pt[s, b], 1].transpose(1, 0, 2)
+            k_ref = c.k[0][32 * b:32 * (b + 1)]
+            tol = 1e-6 if dtype == "f32" else 2.0 ** -8 * np.abs(k_ref) + 1e-6
+            assert np.all(np.abs(k_gpu - k_ref) <= tol)
+            np.testing.assert_array_equal(v_gpu, c.v[0][32 * b:32 * (b + 1)])
+
+
+def test_commit_bulk_equals_block_by_block():
+    from decoding_bd_block_b200 import bd
+    from decoding_bd_block_b200.step import BlockCacheState, to_device
+    cfg = dataclasses.replace(W.QWEN15B_STEP, batch=2, seed=78)
+    P = np.array([256, 128])
+    a = W.make_attn_inputs(cfg, P)
+    bulk = BlockCacheState(cfg, P, a["prefix_k"], a["prefix_v"])
+    one = BlockCacheState(cfg, P, None, None)
+    for s in range(2):
+        for b in range(P[s] // 32):
+            k = to_device(a["prefix_k"][s][32 * b:32 * (b + 1)], cfg.dtype)
+            v = to_device(a["prefix_v"][s][32 * b:32 * (b + 1)], cfg.dtype)
+            bd.bd_cache_commit(one.cache, k, v, [s], 1)
+    torch.cuda.synchronize()
+    for s in range(2):
+        for b in range(P[s] // 32):
+            pb = bulk.cache.page_table_host[s, b]
+            po = one.cache.page_table_host[s, b]
+            assert torch.equal(bulk.cache.pages[pb], one.cache.pages[po])
+
+
+# --------------------------------------------------------- block attention
+ATTN_CASES = [
+    W.TINY_F32,
+    W.QWEN15B_STEP,
+    W.QWEN7B_RAGGED,
+    dataclasses.replace(W.TINY_F32, name="f32_d128_ragged", head_dim=128, batch=3,
+                        prefix_tokens=(0, 32, 640), seed=91),
+    dataclasses.replace(W.QWEN15B_STEP, name="bf16_d64_empty_prefix", head_dim=64,
+                        prefix_tokens=(0,), seed=92),
+    dataclasses.replace(W.QWEN7B_RAGGED, name="bf16_g7_long_ragged", batch=3,
+                        prefix_range=(), prefix_tokens=(4096, 32, 2080), seed=93),
+]
+
+
+@pytest.mark.parametrize("cfg", ATTN_CASES, ids=lambda c: c.name)
+def test_block_attn_parity(cfg):
+    a, _, step = _step(cfg, sel=False)
+    step.run_attn()
+    torch.cuda.synchronize()
+    got = step.out.float().cpu().numpy()
+    ref = oracle_block_attn(cfg, a)
+    err = max(float(np.abs(got[s] - ref[s]).max()) for s in ref)
+    assert err <= ATOL[cfg.dtype], err
+
+
+def test_block_attn_longctx_sampled():
+    cfg = W.LONGCTX_ATTN
+    a, _, step = _step(cfg, sel=False)
+    step.run_attn()
+    torch.cuda.synchronize()
+    got = step.out.float().cpu().numpy()
+    ref = oracle_block_attn(cfg, a, seqs=[0, 5])
+    for s, r in ref.items():
+        err = float(np.abs(got[s] - r).max())
+        assert err <= ATOL["bf16"], (s, err)
+
+
+def test_block_attn_repeatable_and_after_commit():
+    # The block attention reads n_blocks on the device: commit the current
+    # block, attend again with a new block, compare with the oracle.
+    from decoding_bd_block_b200 import bd
+    cfg = dataclasses.replace(W.TINY_F32, batch=2, prefix_tokens=(64, 0), seed=94)
+    a, _, step = _step(cfg, sel=False)
+    step.run_attn()
+    first = step.out.clone()
+    step.run_attn()
+    torch.cuda.synchronize()
+    assert torch.equal(first, step.out)
+    bd.bd_cache_commit(step.cstate.cache, step.k_blk, step.v_blk, [0, 1], 1)
+    a2 = W.make_attn_inputs(dataclasses.replace(cfg, seed=95), np.array([96, 32]))
+    for key in ("prefix_k", "prefix_v"):
+        a2[key] = [np.concatenate([a[key][s], a[{"prefix_k": "k_blk", "prefix_v": "v_blk"}[key]][s]])
+                   for s in range(2)]
+    from decoding_bd_block_b200.step import to_device
+    step.q.copy_(to_device(a2["q"], cfg.dtype))
+    step.k_blk.copy_(to_device(a2["k_blk"], cfg.dtype))
+    step.v_blk.copy_(to_device(a2["v_blk"], cfg.dtype))
+    n = bd.bd_block_attn_workspace_size(step.cstate.cache)
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device="cuda")
+    bd.bd_block_attn(step.cstate.cache, step.q, step.k_blk, step.v_blk, step.out, ws)
+    torch.cuda.synchronize()
+    ref = oracle_block_attn(cfg, a2)
+    got = step.out.cpu().numpy()
+    assert max(float(np.abs(got[s] - ref[s]).max()) for s in ref) <= ATOL["f32"]
+
+
+# ---------------------------------------------------- confidence select
+SELECT_CASES = [
+    (W.TINY_F32, 0.9, 8), (W.TINY_F32, 1.0, 8), (W.TINY_F32, 0.9, 32), (W.TINY_F32, 1.0, 32),
+    (W.TINY_F32_LITERAL, 0.9, 8),
+    (W.QWEN15B_STEP, 0.9, 8),
+    (W.QWEN7B_RAGGED, 0.9, 8),
+    (W.QWEN7B_RAGGED, 0.9, 32),
+    (dataclasses.replace(W.QWEN15B_STEP, name="bf16_vocab_tail", vocab=1000, hidden=512, batch=5,
+                         n_masked=0, masked_range=(0, 32), seed=96), 0.5, 4),
+    (dataclasses.replace(W.TINY_F32, name="f32_all_masked_tau0", batch=4, n_masked=32,
+                         seed=97), 0.0, 8),
+    (dataclasses.replace(W.TINY_F32, name="f32_subblock1", batch=4, n_masked=0,
+                         masked_range=(0, 32), seed=98), 0.9, 1),
+]
+
+
+@pytest.mark.parametrize("case", SELECT_CASES, ids=lambda c: f"{c[0].name}-tau{c[1]}-S{c[2]}")
+def test_confidence_select_parity(case):
+    cfg, tau, S = case
+    _, s, step = _step(cfg, attn=False)
+    step.run_select(tau, S)
+    torch.cuda.synchronize()
+    ref = O.confidence_select(s["h"], s["h_prev"], s["W"], s["masked_bits"], tau, S,
+                              s["tokens"], cfg.dtype)
+    res = compare_select(ref, step.tokens.cpu().numpy(), step.unmask.cpu().numpy().view(np.uint32),
+                         step.pmax.cpu().numpy(), step.argmax.cpu().numpy(), s["masked_bits"])
+    print(cfg.name, tau, S, res)
+    if tau == 1.0:
+        for b in range(cfg.batch):
+            want = 1 if s["masked_bits"][b] else 0
+            assert bin(int(step.unmask[b].item()) & 0xFFFFFFFF).count("1") == want
+
+
+def test_select_idempotent_and_masked_untouched():
+    cfg = dataclasses.replace(W.QWEN15B_STEP, batch=3, vocab=4096, seed=99)
+    _, s, step = _step(cfg, attn=False)
+    step.run_select(0.9, 8)
+    t1, u1 = step.tokens.clone(), step.unmask.clone()
+    step.run_select(0.9, 8)
+    torch.cuda.synchronize()
+    assert torch.equal(t1, step.tokens) and torch.equal(u1, step.unmask)
+    assert torch.equal(step.masked.cpu(), torch.from_numpy(s["masked_bits"].view(np.int32)))
+    tin = step.tokens_in.cpu().numpy()
+    tout = step.tokens.cpu().numpy()
+    un = step.unmask.cpu().numpy().view(np.uint32)
+    for b in range(3):
+        for i in range(32):
+            if not (int(un[b]) >> i) & 1:
+                assert tout[b, i] == tin[b, i]
+
+
+# -------------------------------------------------- 2L x 2L mask attention
+def _mask_case(L, D, dtype, n=2, Hq=4, Hkv=2, d=64, seed=5):
+    cfg = W.MaskAttnConfig(name="t", samples=n, views=2, L=L, block=D, n_heads_q=Hq,
+                           n_heads_kv=Hkv, head_dim=d, seed=seed, dtype=dtype)
+    return cfg, W.make_mask_attn_inputs(cfg)
+
+
+def _run_mask(cfg, t):
+    from decoding_bd_block_b200 import bd
+    from decoding_bd_block_b200.step import to_device
+    q, k, v = (to_device(t[x], cfg.dtype) for x in ("q", "k", "v"))
+    out = torch.empty_like(q)
+    shape = bd.make_shape(cfg.n_heads_q, cfg.n_heads_kv, cfg.head_dim, cfg.dtype)
+    bd.bd_block_mask_attn(shape, q, k, v, out, cfg.n_seqs, cfg.L, cfg.block)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("L,D,dtype,d", [(64, 32, "f32", 64), (96, 16, "f32", 128),
+                                         (256, 32, "bf16", 128), (128, 64, "bf16", 64)])
+def test_mask_attn_parity_small(L, D, dtype, d):
+    cfg, t = _mask_case(L, D, dtype, d=d)
+    got = _run_mask(cfg, t)
+    ref = O.mask_attn(O.widen(t["q"], dtype), O.widen(t["k"], dtype), O.widen(t["v"], dtype), L, D)
+    assert float(np.abs(got - ref).max()) <= ATOL[dtype]
+
+
+def test_mask_attn_full_size_sampled():
+    cfg = W.MASK_ATTN
+    t = W.make_mask_attn_inputs(cfg)
+    got = _run_mask(cfg, t)
+    rows = np.arange(0, 2 * cfg.L, 61)
+    for n in (0, 1, cfg.n_seqs - 1):
+        ref = O.mask_attn(O.widen(t["q"][n:n + 1], "bf16"), O.widen(t["k"][n:n + 1], "bf16"),
+                          O.widen(t["v"][n:n + 1], "bf16"), cfg.L, cfg.block, rows=rows)[0]
+        assert float(np.abs(got[n, rows] - ref).max()) <= ATOL["bf16"]
+
+
+# ------------------------------------------------------------ error paths
+def test_host_validation_errors_launch_nothing():
+    from decoding_bd_block_b200 import bd
+    from decoding_bd_block_b200.step import BlockCacheState, to_device
+    cfg = dataclasses.replace(W.TINY_F32, batch=2, seed=100)
+    st = BlockCacheState(cfg, np.array([32, 32]), None, None, extra_blocks=0)
+    k = to_device(np.zeros((1, 64, 2, 64), np.float32), "f32")
+    with pytest.raises(bd.BdError) as e:            # 2 blocks > max_blocks = 1
+        bd.bd_cache_commit(st.cache, k, k, [0], 2)
+    assert e.value.status == -3
+    with pytest.raises(bd.BdError) as e:            # repeated sequence
+        bd.bd_cache_commit(st.cache, k, k, [1, 1], 1)
+    assert e.value.status == -1
+    st.cache.page_table_host[1, 0] = st.cache.page_table_host[0, 0]
+    bd.bd_cache_commit(st.cache, k[:, :32], k[:, :32], [0], 1)
+    with pytest.raises(bd.BdError) as e:            # page already holds a block
+        bd.bd_cache_commit(st.cache, k[:, :32], k[:, :32], [1], 1)
+    assert e.value.status == -1
+    assert list(st.cache.n_blocks_host) == [1, 0]
+    a = W.make_attn_inputs(cfg, np.array([32, 0]))
+    q = to_device(a["q"], "f32")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(bd.BdError) as e:
+        bd.bd_block_attn(st.cache, q, q, q, torch.empty_like(q), ws, workspace_bytes=0)
+    assert e.value.status == -4
