@@ -36,7 +36,7 @@ from decoding_bd_block_b200 import workloads as W  # noqa: E402
 DEFAULT_WORKLOAD = W.QWEN15B_STEP.name
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
-SELECT_KERNEL_SOURCES = ("decoding_bd_block_b200/csrc/select_simt.cu",)
+SELECT_KERNEL_SOURCES = ("decoding_bd_block_b200/csrc/select_tc.cu", "decoding_bd_block_b200/csrc/tc_common.cuh")
 
 
 def parse_args(argv=None):

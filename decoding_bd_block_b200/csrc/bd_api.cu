@@ -161,6 +161,10 @@ int bd_confidence_select(int32_t dtype, int32_t batch, int32_t hidden, int32_t v
   if (dtype != BD_F32 && dtype != BD_BF16) return BD_ERR_UNSUPPORTED;
   if (hidden % 8 != 0) return BD_ERR_UNSUPPORTED;
   if (!h || !h_prev || !w || !masked_bits || !tokens || !unmask_bits) return BD_ERR_INVALID_ARG;
+  // rows are copied in 16-byte vectors and W is read by TMA
+  if ((reinterpret_cast<uintptr_t>(h) | reinterpret_cast<uintptr_t>(h_prev) |
+       reinterpret_cast<uintptr_t>(w)) % 16 != 0)
+    return BD_ERR_INVALID_ARG;
   if (sub_block <= 0 || sub_block > bd::kBlock || bd::kBlock % sub_block != 0)
     return BD_ERR_INVALID_ARG;
   if (!(tau >= 0.f)) return BD_ERR_INVALID_ARG;

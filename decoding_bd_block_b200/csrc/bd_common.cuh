@@ -115,10 +115,17 @@ cudaError_t launch_block_attn(const bd_attn_shape& sh, const bd_kv_cache& c, con
                               const void* q, const void* k, const void* v, void* out, void* ws,
                               cudaStream_t st);
 
+// Tensor-core LM head (select_tc.cu): persistent grid size and launcher.
+int lmhead_tc_grid();
+cudaError_t launch_lmhead_tc(const void* rows, const void* w, const int32_t* count, int H, int V,
+                             int rows_alloc, int part_stride, float* pm, float* ps, int32_t* pa,
+                             int32_t* status, cudaStream_t st);
+
 struct SelectPlan {
+  bool tc;           // LM head on tcgen05 (bf16)
   int n_split;       // vocab splits (partials per row)
   int rows_alloc;    // packed-row capacity (>= 32 * batch, padded)
-  size_t off_rows, off_rowmap, off_posrow, off_count, off_pm, off_ps, off_pa, total;
+  size_t off_rows, off_posrow, off_count, off_pm, off_ps, off_pa, total;
 };
 SelectPlan plan_confidence_select(int dtype, int batch, int hidden, int vocab);
 cudaError_t launch_confidence_select(int dtype, int batch, int hidden, int vocab,

@@ -4,60 +4,63 @@
 //
 // Launches:
 //   1. gather_rows     packs, per masked position i, hidden row i-1 (h_prev
-//                      for i = 0) into a dense [M][H] matrix; records the
-//                      row of each position and M;
-//   2. lm head stats   vocab-split: each CTA folds its vocab range into a
+//                      for i = 0) into a dense [M][H] matrix (one warp per
+//                      position, 16-byte copies); records each position's
+//                      row and M;
+//   2. LM-head stats   vocab-split: each CTA folds its vocab range into a
 //                      running (max, sum exp, argmax) per row; logits stay on
-//                      chip (CUDA-core tile here, tcgen05 in select_tc.cu);
-//   3. merge_select    merges the partials of every row, turns them into
-//                      p_max and the token, and applies the unmask rule.
+//                      chip (tcgen05 in select_tc.cu for bf16; the CUDA-core
+//                      tile below for fp32);
+//   3. merge_select    one warp per position merges that row's partials,
+//                      turns them into p_max and the token; warp 0 then
+//                      applies the unmask rule of the sequence.
+// Partials are stored [row][part] so a row's partials are contiguous.
 #include "bd_common.cuh"
 
 namespace bd {
 
-// grid (batch), 256 threads.
+// grid (batch), 1024 threads: warp i copies the row of position i.
 template <typename T>
-__global__ void __launch_bounds__(256) gather_rows_kernel(
+__global__ void __launch_bounds__(1024) gather_rows_kernel(
     const T* __restrict__ h, const T* __restrict__ h_prev, const uint32_t* __restrict__ masked,
-    int B, int H, T* __restrict__ rows, int32_t* __restrict__ rowmap,
-    int32_t* __restrict__ posrow, int32_t* __restrict__ count, int rows_alloc) {
-  __shared__ int red[8];
+    int B, int H, T* __restrict__ rows, int32_t* __restrict__ posrow,
+    int32_t* __restrict__ count, int rows_alloc) {
+  __shared__ int red[32];
   const int s = blockIdx.x;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   int acc = 0;
   for (int x = threadIdx.x; x < s; x += blockDim.x) acc += __popc(masked[x]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = acc;
+  if (lane == 0) red[warp] = acc;
   __syncthreads();
   int off = 0;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) off += red[w];
+  for (int w = 0; w < 32; ++w) off += red[w];
   const uint32_t bits = masked[s];
-  if (threadIdx.x < kBlock) {
-    const int i = threadIdx.x;
-    int r = -1;
-    if ((bits >> i) & 1u) {
-      r = off + __popc(bits & ((1u << i) - 1u));
-      rowmap[r] = s * kBlock + i;
-    }
-    posrow[s * kBlock + i] = r;
-  }
-  int k = 0;
-  for (int i = 0; i < kBlock; ++i) {
-    if (!((bits >> i) & 1u)) continue;
+  const int i = warp;
+  const bool is_m = (bits >> i) & 1u;
+  const int r = is_m ? off + __popc(bits & ((1u << i) - 1u)) : -1;
+  if (lane == 0) posrow[s * kBlock + i] = r;
+  if (is_m) {
     const T* src = (i == 0) ? h_prev + static_cast<size_t>(s) * H
                             : h + (static_cast<size_t>(s) * kBlock + i - 1) * H;
-    T* dst = rows + static_cast<size_t>(off + k) * H;
-    for (int x = threadIdx.x; x < H; x += blockDim.x) dst[x] = src[x];
-    ++k;
+    T* dst = rows + static_cast<size_t>(r) * H;
+    const int nvec = H * static_cast<int>(sizeof(T)) / 16;  // H * sizeof(T) % 16 == 0
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    for (int x = lane; x < nvec; x += 32) d4[x] = s4[x];
   }
   if (s == B - 1) {
     const int total = off + __popc(bits);
-    if (threadIdx.x == 0) *count = total;
+    if (threadIdx.x == 0) {
+      count[0] = total;
+      count[1] = 0;  // status word of the LM-head kernel
+    }
     const int pad_end = min(rows_alloc, (total + 15) / 16 * 16);
-    for (size_t x = static_cast<size_t>(total) * H + threadIdx.x;
-         x < static_cast<size_t>(pad_end) * H; x += blockDim.x)
-      rows[x] = from_f32<T>(0.f);
+    const int nvec = (pad_end - total) * H * static_cast<int>(sizeof(T)) / 16;
+    uint4* d4 = reinterpret_cast<uint4*>(rows + static_cast<size_t>(total) * H);
+    for (int x = threadIdx.x; x < nvec; x += blockDim.x) d4[x] = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -66,7 +69,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(
 template <typename T>
 __global__ void __launch_bounds__(256) lmhead_simt_kernel(
     const T* __restrict__ rows, const T* __restrict__ w, const int32_t* __restrict__ count,
-    int H, int V, int n_split, int rows_alloc, float* __restrict__ pm, float* __restrict__ ps,
+    int H, int V, int n_split, float* __restrict__ pm, float* __restrict__ ps,
     int32_t* __restrict__ pa) {
   __shared__ float Ws[32][68];
   __shared__ float Rs[32][36];
@@ -126,34 +129,62 @@ __global__ void __launch_bounds__(256) lmhead_simt_kernel(
     }
   }
   if (tid < 32 && r0 + tid < M) {
-    const size_t idx = static_cast<size_t>(blockIdx.x) * rows_alloc + r0 + tid;
+    const size_t idx = static_cast<size_t>(r0 + tid) * n_split + blockIdx.x;
     pm[idx] = run_m;
     ps[idx] = run_s;
     pa[idx] = run_a;
   }
 }
 
-// grid (batch), 32 threads: thread i owns position i of sequence s.
-__global__ void __launch_bounds__(32) merge_select_kernel(
-    const int32_t* __restrict__ posrow, const uint32_t* __restrict__ masked, int n_split,
-    int rows_alloc, const float* __restrict__ pm, const float* __restrict__ ps,
-    const int32_t* __restrict__ pa, float tau, int S, int32_t* __restrict__ tokens,
-    uint32_t* __restrict__ unmask, float* __restrict__ pmax_out, int32_t* __restrict__ argmax_out) {
-  const int s = blockIdx.x, i = threadIdx.x;
+// grid (batch), 1024 threads: warp i merges the partials of position i.
+// With grouped partials (tensor-core LM head) each row has n_split / G
+// parts, G = ceil(M / 256) row groups.  A nonzero status word (a bounded
+// wait gave up) turns the outputs into "no decision": nothing is unmasked,
+// p_max is NaN and the token -2.
+__global__ void __launch_bounds__(1024) merge_select_kernel(
+    const int32_t* __restrict__ posrow, const int32_t* __restrict__ count,
+    const uint32_t* __restrict__ masked, int n_split, int grouped, const float* __restrict__ pm,
+    const float* __restrict__ ps, const int32_t* __restrict__ pa, float tau, int S,
+    int32_t* __restrict__ tokens, uint32_t* __restrict__ unmask, float* __restrict__ pmax_out,
+    int32_t* __restrict__ argmax_out) {
+  __shared__ float sp[kBlock];
+  __shared__ int stok[kBlock];
+  const int s = blockIdx.x;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t bits = masked[s];
-  const bool is_m = (bits >> i) & 1u;
-  float p = 0.f;
-  int tok = -1;
-  if (is_m) {
-    const int r = posrow[s * kBlock + i];
-    Stat st = stat_empty();
-    for (int k = 0; k < n_split; ++k) {
-      const size_t idx = static_cast<size_t>(k) * rows_alloc + r;
-      st = stat_combine(st, Stat{pm[idx], ps[idx], pa[idx]});
+  if (count[1] != 0) {
+    if (threadIdx.x < kBlock) {
+      if (threadIdx.x == 0) unmask[s] = 0u;
+      if (pmax_out) pmax_out[s * kBlock + threadIdx.x] = __int_as_float(0x7fc00000);
+      if (argmax_out) argmax_out[s * kBlock + threadIdx.x] = -2;
     }
-    p = 1.f / st.s;
-    tok = st.a;
+    return;
   }
+  const int parts = grouped ? n_split / ((count[0] + 255) / 256) : n_split;
+  {
+    const int i = warp;
+    Stat st = stat_empty();
+    if ((bits >> i) & 1u) {
+      const size_t base = static_cast<size_t>(posrow[s * kBlock + i]) * n_split;
+      for (int k = lane; k < parts; k += 32) st = stat_combine(st, Stat{pm[base + k], ps[base + k], pa[base + k]});
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const Stat other{__shfl_xor_sync(0xffffffffu, st.m, o), __shfl_xor_sync(0xffffffffu, st.s, o),
+                         __shfl_xor_sync(0xffffffffu, st.a, o)};
+        st = stat_combine(st, other);
+      }
+    }
+    if (lane == 0) {
+      sp[i] = st.s > 0.f ? 1.f / st.s : 0.f;
+      stok[i] = st.a;
+    }
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  const int i = lane;
+  const bool is_m = (bits >> i) & 1u;
+  const float p = is_m ? sp[i] : 0.f;
+  const int tok = is_m ? stok[i] : -1;
   // Candidates: masked positions of the lowest sub-block that has one.
   const int first = bits ? __ffs(static_cast<int>(bits)) - 1 : 0;
   const int k0 = (first / S) * S;
@@ -181,25 +212,34 @@ __global__ void __launch_bounds__(32) merge_select_kernel(
 }
 
 // -------------------------------------------------------------- host side
+// The tensor-core LM head takes bf16 whenever every row group of <= 256 rows
+// still gets at least one vocab range of its own.
+static bool use_tc(int dtype, int batch) {
+  return dtype == BD_BF16 && (batch * kBlock + 255) / 256 <= lmhead_tc_grid();
+}
+
 SelectPlan plan_confidence_select(int dtype, int batch, int hidden, int vocab) {
   SelectPlan p{};
   p.rows_alloc = static_cast<int>(align_up(static_cast<size_t>(batch) * kBlock, 256));
-  const int vtiles = (vocab + 63) / 64;
-  const int rtiles = p.rows_alloc / 32;
-  int ns = (4 * 148 + rtiles - 1) / rtiles;
-  if (ns > vtiles) ns = vtiles;
-  if (ns < 1) ns = 1;
-  p.n_split = ns;
+  p.tc = use_tc(dtype, batch);
+  if (p.tc) {
+    p.n_split = lmhead_tc_grid();
+  } else {
+    const int vtiles = (vocab + 63) / 64;
+    const int rtiles = p.rows_alloc / 32;
+    int ns = (4 * 148 + rtiles - 1) / rtiles;
+    if (ns > vtiles) ns = vtiles;
+    if (ns < 1) ns = 1;
+    p.n_split = ns;
+  }
   const size_t es = dtype == BD_BF16 ? 2 : 4;
   size_t off = 0;
   p.off_rows = off;
   off = align_up(off + static_cast<size_t>(p.rows_alloc) * hidden * es, 256);
-  p.off_rowmap = off;
-  off = align_up(off + static_cast<size_t>(p.rows_alloc) * 4, 256);
   p.off_posrow = off;
   off = align_up(off + static_cast<size_t>(batch) * kBlock * 4, 256);
-  p.off_count = off;
-  off = align_up(off + 4, 256);
+  p.off_count = off;  // [0] = M, [1] = status word of the tensor-core kernel
+  off = align_up(off + 8, 256);
   const size_t part = static_cast<size_t>(p.n_split) * p.rows_alloc * 4;
   p.off_pm = off;
   off = align_up(off + part, 256);
@@ -219,20 +259,28 @@ static cudaError_t launch_select_t(int batch, int hidden, int vocab, const Selec
                                    void* ws, cudaStream_t st) {
   char* base = static_cast<char*>(ws);
   T* rows = reinterpret_cast<T*>(base + p.off_rows);
-  int32_t* rowmap = reinterpret_cast<int32_t*>(base + p.off_rowmap);
   int32_t* posrow = reinterpret_cast<int32_t*>(base + p.off_posrow);
   int32_t* count = reinterpret_cast<int32_t*>(base + p.off_count);
   float* pm = reinterpret_cast<float*>(base + p.off_pm);
   float* ps = reinterpret_cast<float*>(base + p.off_ps);
   int32_t* pa = reinterpret_cast<int32_t*>(base + p.off_pa);
-  gather_rows_kernel<T><<<batch, 256, 0, st>>>(static_cast<const T*>(h),
-                                               static_cast<const T*>(h_prev), masked, batch,
-                                               hidden, rows, rowmap, posrow, count, p.rows_alloc);
-  lmhead_simt_kernel<T><<<dim3(p.n_split, p.rows_alloc / 32), 256, 0, st>>>(
-      rows, static_cast<const T*>(w), count, hidden, vocab, p.n_split, p.rows_alloc, pm, ps, pa);
-  merge_select_kernel<<<batch, 32, 0, st>>>(posrow, masked, p.n_split, p.rows_alloc, pm, ps, pa,
-                                            tau, S, tokens, unmask, pmax_out, argmax_out);
-  count_launches(3);
+  gather_rows_kernel<T><<<batch, 1024, 0, st>>>(static_cast<const T*>(h),
+                                                static_cast<const T*>(h_prev), masked, batch,
+                                                hidden, rows, posrow, count, p.rows_alloc);
+  count_launches(1);
+  if (p.tc) {
+    const cudaError_t e = launch_lmhead_tc(rows, w, count, hidden, vocab, p.rows_alloc, p.n_split,
+                                           pm, ps, pa, count + 1, st);
+    if (e != cudaSuccess) return e;
+  } else {
+    lmhead_simt_kernel<T><<<dim3(p.n_split, p.rows_alloc / 32), 256, 0, st>>>(
+        rows, static_cast<const T*>(w), count, hidden, vocab, p.n_split, pm, ps, pa);
+    count_launches(1);
+  }
+  merge_select_kernel<<<batch, 1024, 0, st>>>(posrow, count, masked, p.n_split, p.tc ? 1 : 0,
+                                              pm, ps, pa, tau, S, tokens, unmask, pmax_out,
+                                              argmax_out);
+  count_launches(1);
   return cudaGetLastError();
 }
 

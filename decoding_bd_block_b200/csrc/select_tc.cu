@@ -1,0 +1,303 @@
+// LM-head statistics on the 5th-generation tensor cores (bf16 in, fp32
+// accumulate), for bd_confidence_select.
+//
+// Each packed row r (the hidden row that predicts one masked position) needs
+// max_v l, sum_v exp(l - max) and argmax_v of l = row . W[v] over the whole
+// vocabulary ("Fast-dLLM v2: Efficient Block-Diffusion LLM", key design 3:
+// confidence of a masked token; Fast-dLLM v1 article, core technique 2).
+// The logits never leave the chip:
+//
+//   * W is the MMA's M operand: one 128-row vocab tile per accumulator, its
+//     K-slices (64 hidden elements, 16 KB) streamed by TMA through a ring of
+//     shared-memory stages; the packed rows are the N operand (N <= 256).
+//   * Persistent CTAs: rows are split into G groups of <= 256 (G = 1 for
+//     M <= 256); the vocab tiles into R = gridDim / G contiguous ranges; CTA
+//     (group, range) streams its range once.
+//   * Warp roles: warp 0 issues TMA, warp 1 issues tcgen05.mma into one of
+//     two TMEM accumulators (128 lanes x 256 fp32 columns each), warps 2-5
+//     drain the other accumulator: per column (= packed row) a warp-wide
+//     max / argmax / sum of exp over its 32 vocab lanes, folded into a
+//     running (max, sum, argmax) that lane (column mod 32) keeps.
+//   * At the end the 4 epilogue warps combine through shared memory and the
+//     CTA writes one (max, sum, argmax) partial per row of its group.
+#include "bd_common.cuh"
+#include "tc_common.cuh"
+
+namespace bd {
+namespace {
+
+constexpr int kThreads = 192;      // 6 warps
+constexpr int kVTile = 128;        // vocab rows per MMA (M)
+constexpr int kKStage = 64;        // hidden elements per stage (128 B rows)
+constexpr int kMaxN = 256;         // packed rows per group (MMA N)
+constexpr int kMaxStages = 12;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kWBytes = kVTile * kKStage * 2;  // 16 KB
+constexpr int kSmemBytes = 200 * 1024;  // + ~12.5 KB static stays under 227 KB
+
+struct SelectTcArgs {
+  const int32_t* count;  // M (written by the gather kernel)
+  int H, V;
+  int rows_alloc;
+  int part_stride;  // partials are [row][part]
+  float* pm;
+  float* ps;
+  int32_t* pa;
+  int32_t* status;
+};
+
+__device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
+                     const __grid_constant__ CUtensorMap tm_rows, SelectTcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle atoms.
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  __shared__ uint64_t full_bar[kMaxStages], empty_bar[kMaxStages];
+  __shared__ uint64_t tfull_bar[2], tempty_bar[2];
+  __shared__ uint32_t tmem_slot;
+  __shared__ float red_m[4][kMaxN];
+  __shared__ float red_s[4][kMaxN];
+  __shared__ int red_a[4][kMaxN];
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int M = *a.count;
+  if (M <= 0) return;
+  const int G = (M + kMaxN - 1) / kMaxN;
+  const int R = gridDim.x / G;
+  const int group = blockIdx.x / R, range = blockIdx.x % R;
+  if (group >= G) return;
+  const int Ng = round16((M + G - 1) / G);
+  const int row0 = group * Ng;
+  const int rows_here = min(Ng, M - row0);
+  if (rows_here <= 0) return;
+  const int N = round16(rows_here);
+  const int n_vt = (a.V + kVTile - 1) / kVTile;
+  const int t0 = static_cast<int>(static_cast<long long>(range) * n_vt / R);
+  const int t1 = static_cast<int>(static_cast<long long>(range + 1) * n_vt / R);
+  const int n_k = (a.H + kKStage - 1) / kKStage;
+  const int b_bytes = N * kKStage * 2;
+  const int stage_bytes = (kWBytes + b_bytes + 1023) & ~1023;
+  int n_stages = (kSmemBytes - 1024) / stage_bytes;
+  n_stages = n_stages > kMaxStages ? kMaxStages : n_stages;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < n_stages; ++s) {
+      tc::mbar_init(&full_bar[s], 1);
+      tc::mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&tfull_bar[b], 1);
+      tc::mbar_init(&tempty_bar[b], 4);
+    }
+    tc::fence_barrier_init();
+    tc::fence_proxy_async();
+  }
+  if (warp == 1) tc::tmem_alloc(&tmem_slot, kTmemCols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_w);
+      tc::prefetch_tmap(&tm_rows);
+      const uint64_t pol_w = tc::policy_evict_first();
+      const uint64_t pol_r = tc::policy_evict_last();
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = t0; t < t1 && ok; ++t) {
+        for (int kb = 0; kb < n_k; ++kb) {
+          if (!tc::mbar_wait(&empty_bar[s], ph ^ 1, a.status)) { ok = false; break; }
+          uint8_t* st = smem + static_cast<size_t>(s) * stage_bytes;
+          tc::mbar_arrive_expect_tx(&full_bar[s], kWBytes + b_bytes);
+          tc::tma_load_2d(st, &tm_w, &full_bar[s], kb * kKStage, t * kVTile, pol_w);
+          for (int j = 0; j < N / 16; ++j)
+            tc::tma_load_2d(st + kWBytes + j * 2048, &tm_rows, &full_bar[s], kb * kKStage,
+                            row0 + 16 * j, pol_r);
+          if (++s == n_stages) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16_f32(kVTile, N);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = t0, it = 0; t < t1 && ok; ++t, ++it) {
+        const int b = it & 1;
+        const uint32_t tph = (it >> 1) & 1;
+        if (!tc::mbar_wait(&tempty_bar[b], tph ^ 1, a.status)) break;
+        tc::tc_fence_after();
+        const uint32_t d = tmem + b * kMaxN;
+        for (int kb = 0; kb < n_k; ++kb) {
+          if (!tc::mbar_wait(&full_bar[s], ph, a.status)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t sa = tc::smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+          const uint32_t sb = sa + kWBytes;
+#pragma unroll
+          for (int kk = 0; kk < kKStage / 16; ++kk)
+            tc::mma_bf16_ss(d, tc::sdesc_kmajor_sw128(sa + kk * 32),
+                            tc::sdesc_kmajor_sw128(sb + kk * 32), idesc, (kb | kk) != 0);
+          tc::mma_commit(&empty_bar[s]);
+          if (++s == n_stages) { s = 0; ph ^= 1; }
+        }
+        tc::mma_commit(&tfull_bar[b]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    float run_m[8], run_s[8];
+    int run_a[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      run_m[c] = -INFINITY;
+      run_s[c] = 0.f;
+      run_a[c] = 0x7fffffff;
+    }
+    const int n_chunks = N / 32 + ((N % 32) ? 1 : 0);
+    bool ok = true;
+    for (int t = t0, it = 0; t < t1 && ok; ++t, ++it) {
+      const int b = it & 1;
+      const uint32_t tph = (it >> 1) & 1;
+      if (!tc::mbar_wait(&tfull_bar[b], tph, a.status)) { ok = false; break; }
+      tc::tc_fence_after();
+      const int v = t * kVTile + q * 32 + lane;  // vocab row of this thread's lane
+      const bool v_ok = v < a.V;
+      const int vbase = t * kVTile + q * 32;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        if (c < n_chunks) {
+          uint32_t r[32];
+          tc::tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + b * kMaxN + c * 32,
+                                 r);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float x = v_ok ? __uint_as_float(r[j]) : -INFINITY;
+            const float mx = tc::redux_max_f32(x);
+            if (mx == -INFINITY) continue;  // warp-uniform
+            const uint32_t bal = __ballot_sync(0xffffffffu, x == mx);
+            const int arg = vbase + __ffs(bal) - 1;
+            float e = fast_exp2((x - mx) * kLog2e);
+            e += __shfl_xor_sync(0xffffffffu, e, 16);
+            e += __shfl_xor_sync(0xffffffffu, e, 8);
+            e += __shfl_xor_sync(0xffffffffu, e, 4);
+            e += __shfl_xor_sync(0xffffffffu, e, 2);
+            e += __shfl_xor_sync(0xffffffffu, e, 1);
+            if (lane == j) {
+              if (mx > run_m[c]) {
+                run_s[c] = run_s[c] * fast_exp2((run_m[c] - mx) * kLog2e) + e;
+                run_m[c] = mx;
+                run_a[c] = arg;
+              } else {
+                run_s[c] += e * fast_exp2((mx - run_m[c]) * kLog2e);
+                if (mx == run_m[c] && arg < run_a[c]) run_a[c] = arg;
+              }
+            }
+          }
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty_bar[b]);
+    }
+    // combine the 4 lane quarters through shared memory
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int col = c * 32 + lane;
+      if (col < N) {
+        red_m[q][col] = run_m[c];
+        red_s[q][col] = run_s[c];
+        red_a[q][col] = run_a[c];
+      }
+    }
+    tc::named_bar_sync(1, 128);
+    const int et = threadIdx.x - 64;
+    for (int col = et; col < rows_here; col += 128) {
+      Stat st = stat_empty();
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) st = stat_combine(st, Stat{red_m[qq][col], red_s[qq][col], red_a[qq][col]});
+      const size_t idx = static_cast<size_t>(row0 + col) * a.part_stride + range;
+      a.pm[idx] = st.m;
+      a.ps[idx] = st.s;
+      a.pa[idx] = st.a;
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (row-major), tile box [box_rows][64 cols],
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+int lmhead_tc_grid() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+
+cudaError_t launch_lmhead_tc(const void* rows, const void* w, const int32_t* count, int H, int V,
+                             int rows_alloc, int part_stride, float* pm, float* ps, int32_t* pa,
+                             int32_t* status, cudaStream_t st) {
+  CUtensorMap tm_w, tm_rows;
+  if (!make_tmap_2d(&tm_w, w, static_cast<uint64_t>(V), static_cast<uint64_t>(H), kVTile) ||
+      !make_tmap_2d(&tm_rows, rows, static_cast<uint64_t>(rows_alloc), static_cast<uint64_t>(H),
+                    16))
+    return cudaErrorInvalidValue;
+  SelectTcArgs a{count, H, V, rows_alloc, part_stride, pm, ps, pa, status};
+  cudaFuncSetAttribute(lmhead_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       kSmemBytes + 1024);
+  lmhead_tc_kernel<<<lmhead_tc_grid(), kThreads, kSmemBytes + 1024, st>>>(tm_w, tm_rows, a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace bd

@@ -158,8 +158,12 @@ BD_API int bd_block_attn(const bd_attn_shape* shape, const bd_kv_cache* cache,
  *                position, NaN elsewhere
  *   argmax_out   device, [batch][32] int32 or NULL: token per masked
  *                position, -1 elsewhere
- * sub_block must divide 32; 0 <= tau.  Workspace: see
- * bd_confidence_select_workspace_size(). */
+ * sub_block must divide 32; 0 <= tau; hidden % 8 == 0; h, h_prev and w_lm
+ * 16-byte aligned.  Workspace: bd_confidence_select_workspace_size() bytes,
+ * 256-byte aligned.  bf16 runs the LM head on the tensor cores (tcgen05):
+ * if one of its bounded waits ever gives up (it never should), the call
+ * reports "no decision" for the whole batch: unmask_bits 0, p_max NaN and
+ * argmax -2. */
 BD_API int bd_confidence_select_workspace_size(int32_t dtype, int32_t batch,
                                         int32_t hidden, int32_t vocab,
                                         size_t* bytes);

@@ -48,8 +48,10 @@ R7  Selection ([N1] key designs 3 and 4; [N2] item 2; [N4] item 2):
     ([N1] key design 3).  Every masked position of the block is scored.
 R8  Ambiguity: a position's token is ambiguous when its top-2 logit gap is
     < 1e-3; a sequence's unmask decision is ambiguous when some candidate has
-    |p_max - tau| < 1e-4, or when it falls back to the single most confident
-    candidate and the two largest candidate p_max differ by < 1e-4.
+    |p_max - tau| < 1e-4 (only for tau < 1: p_max = 1/Z with Z >= 1 never
+    exceeds 1, so at tau >= 1 the comparison is false on every side), or when
+    it falls back to the single most confident candidate and the two largest
+    candidate p_max differ by < 1e-4.
 """
 from __future__ import annotations
 
@@ -325,7 +327,7 @@ def ambiguity(pmax, gap, masked_bits, tau: float, sub_block: int):
         C = active_candidates(bits, sub_block)
         if not C:
             continue
-        if any(abs(pmax[s][c] - tau) < TAU_EPS for c in C):
+        if tau < 1.0 and any(abs(pmax[s][c] - tau) < TAU_EPS for c in C):
             dec_amb[s] = True
         elif not any(pmax[s][c] > tau for c in C) and len(C) > 1:
             top2 = sorted((pmax[s][c] for c in C), reverse=True)[:2]

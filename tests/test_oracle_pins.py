@@ -351,3 +351,10 @@ def test_ambiguity_flags():
     tok, dec = O.ambiguity(pmax, gap, bits, 0.9, 8)
     np.testing.assert_array_equal(dec, [True, True, False])
     assert tok[0, 1] and not tok[0, 0] and not tok[1].any()
+    # tau = 1: p_max <= 1 can never exceed it, so a saturated p_max near 1 is
+    # no tau-band ambiguity; two saturated candidates still tie in the fallback.
+    p1 = np.full((2, 32), np.nan)
+    p1[0, :2] = [0.99995, 0.5]
+    p1[1, :2] = [0.99999, 0.999991]
+    _, dec1 = O.ambiguity(p1, np.ones((2, 32)), np.array([0b11, 0b11], np.uint32), 1.0, 8)
+    np.testing.assert_array_equal(dec1, [False, True])
