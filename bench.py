@@ -346,7 +346,14 @@ def run_ours(args, cfg, tau, S, dist: Dist):
                     "frac": alg / t_dom / 1e9 / hbm, "traffic": traffic,
                     "algorithmic_bytes_per_launch": alg, "peak_source": peak_kind}
     else:
-        roofline = None
+        es = 2 if cfg.dtype == "bf16" else 4
+        keys = float(np.sum(a_in["prefix_len"] + W.BLOCK))
+        alg = keys * cfg.n_heads_kv * cfg.head_dim * 2 * es
+        t_dom = float(np.mean(t_attn)) / 1e3
+        roofline = {"kernel": "bd_block_attn (K/V stream; whole call timed)", "bound": "hbm",
+                    "achieved": alg / t_dom / 1e9, "peak": hbm, "unit": "GB/s",
+                    "frac": alg / t_dom / 1e9 / hbm, "traffic": recorded_traffic("attn"),
+                    "algorithmic_bytes_per_launch": alg, "peak_source": peak_kind}
 
     e2e = None
     if not args.no_e2e and step.sel:

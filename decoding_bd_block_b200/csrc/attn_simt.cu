@@ -192,6 +192,33 @@ __global__ void __launch_bounds__(D) attn_merge_kernel(const int32_t* __restrict
 }
 
 // -------------------------------------------------------------- host side
+// Tensor-core split: one CTA per SM at a time, so pick the (even) chunk size
+// that minimises waves x (pages per chunk + a fixed cost) over all (chunk, kv
+// head, sequence) CTAs.  The fixed cost, worth ~8 pages of K/V traffic,
+// stands for the CTA's query load (up to 64 KB), set-up and its fp32 partial
+// (m, l, O) for the merge; at least 4 pages (two 64-key stages) per chunk.
+static int plan_tc_chunk(const bd_attn_shape& sh, const bd_kv_cache& c, int max_pages) {
+  int sms = 0, dev = 0;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    sms = 148;
+  const int cap = attn_tc_max_chunk_pages();
+  long long best_cost = -1;
+  int best = cap;
+  for (int ppc = 4; ppc <= cap; ppc += 2) {
+    long long ctas = 0;
+    for (int s = 0; s < c.batch; ++s) ctas += (c.n_blocks_host[s] + 1 + ppc - 1) / ppc;
+    ctas *= sh.n_heads_kv;
+    const long long cost = ((ctas + sms - 1) / sms) * static_cast<long long>(ppc + 8);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = ppc;
+    }
+    if (ppc >= max_pages) break;
+  }
+  return best;
+}
+
 AttnPlan plan_block_attn(const bd_attn_shape& sh, const bd_kv_cache& c) {
   AttnPlan p{};
   long long total_pages = 0;
@@ -200,11 +227,17 @@ AttnPlan plan_block_attn(const bd_attn_shape& sh, const bd_kv_cache& c) {
     total_pages += c.n_blocks_host[s] + 1;
     max_pages = max_pages > c.n_blocks_host[s] + 1 ? max_pages : c.n_blocks_host[s] + 1;
   }
-  // About four CTAs per SM over all (chunk, q head, sequence) work items.
-  const long long target = 4LL * 148;
-  long long ppc = (total_pages * sh.n_heads_q + target - 1) / target;
-  if (ppc < 1) ppc = 1;
-  if (ppc > max_pages) ppc = max_pages;
+  p.tc = attn_tc_supported(sh);
+  long long ppc;
+  if (p.tc) {
+    ppc = plan_tc_chunk(sh, c, max_pages);
+  } else {
+    // About four CTAs per SM over all (chunk, q head, sequence) work items.
+    const long long target = 4LL * 148;
+    ppc = (total_pages * sh.n_heads_q + target - 1) / target;
+    if (ppc < 1) ppc = 1;
+    if (ppc > max_pages) ppc = max_pages;
+  }
   p.pages_per_chunk = static_cast<int>(ppc);
   p.max_chunks = (max_pages + p.pages_per_chunk - 1) / p.pages_per_chunk;
   const size_t es = sh.dtype == BD_BF16 ? 2 : 4;
@@ -219,6 +252,8 @@ AttnPlan plan_block_attn(const bd_attn_shape& sh, const bd_kv_cache& c) {
   off = align_up(off + (p.max_chunks > 1 ? rows * d * 4 : 0), 256);
   p.off_ml = off;
   off = align_up(off + (p.max_chunks > 1 ? rows * 2 * 4 : 0), 256);
+  p.off_status = off;
+  off = align_up(off + 4, 256);
   p.total = off;
   return p;
 }
@@ -235,6 +270,20 @@ static cudaError_t launch_attn_t(const bd_attn_shape& sh, const bd_kv_cache& c, 
   attn_prep_kernel<T><<<dim3(kBlock, c.batch), 128, 0, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), c.n_blocks,
       ws_q, ws_blk, sh.n_heads_q, sh.n_heads_kv, D, sh.rope_theta);
+  count_launches(1);
+  if (p.tc) {
+    const cudaError_t e = launch_attn_tc(sh, c, p.pages_per_chunk, p.max_chunks, ws_q, ws_blk,
+                                         part_o, part_ml, out,
+                                         reinterpret_cast<int32_t*>(w + p.off_status), st);
+    if (e != cudaSuccess) return e;
+    if (p.max_chunks > 1) {
+      attn_merge_kernel<T, D><<<dim3(kBlock, sh.n_heads_q, c.batch), D, 0, st>>>(
+          c.n_blocks, part_o, part_ml, static_cast<T*>(out), sh.n_heads_q, p.pages_per_chunk,
+          p.max_chunks);
+      count_launches(1);
+    }
+    return cudaGetLastError();
+  }
   const size_t smem = (kBlock * D + D * 33 + kBlock * D) * sizeof(float);
   auto kern = attn_split_simt_kernel<T, D>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -246,7 +295,7 @@ static cudaError_t launch_attn_t(const bd_attn_shape& sh, const bd_kv_cache& c, 
     attn_merge_kernel<T, D><<<dim3(kBlock, sh.n_heads_q, c.batch), D, 0, st>>>(
         c.n_blocks, part_o, part_ml, static_cast<T*>(out), sh.n_heads_q, p.pages_per_chunk,
         p.max_chunks);
-  count_launches(p.max_chunks > 1 ? 3 : 2);
+  count_launches(p.max_chunks > 1 ? 2 : 1);
   return cudaGetLastError();
 }
 

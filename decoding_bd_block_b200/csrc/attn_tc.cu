@@ -1,0 +1,421 @@
+// bd_block_attn on the 5th-generation tensor cores (bf16 storage, head_dim
+// 128): the current 32-token block attends to [cached pages ; itself]
+// ("Fast-dLLM v2: Efficient Block-Diffusion LLM", overall framework and key
+// design 3 -- block-internal bidirectional, block-causal across blocks, the
+// finished blocks read from the block-level KV cache).
+//
+// CTA = (split-KV chunk, KV head g, sequence s).  Its query rows are the
+// G = Hq/Hkv heads of group g times the block's 32 positions (row r = head
+// (r / 32) of the group, position r % 32), one or two 128-row tiles Q_t.
+// The chunk's pages stream through a ring of 64-key K/V stages (two pages
+// per stage, TMA with the 128-byte swizzle).  Per stage j and tile t:
+//
+//   warp 1 (one thread)  S_t = Q_t K_j^T   -> TMEM (two 64-column buffers)
+//                        O_t += P_t V_j    (P from shared memory, O in TMEM)
+//   warps 4+4t .. 7+4t   one thread per query row: online softmax in base 2
+//                        (scores pre-scaled by log2(e)/sqrt(d)), P -> bf16
+//                        into shared memory, lazy rescale of its O row in
+//                        TMEM when the running max grows by more than 2^8
+//   warp 0 (one thread)  TMA producer: Q once, then K/V pages
+//
+// The chunk's (m, l, O) go to the workspace for attn_merge_kernel, or --
+// when one chunk covers the whole sequence -- O / l straight to the output.
+#include "bd_common.cuh"
+#include "tc_common.cuh"
+
+namespace bd {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kThreads = 384;               // 12 warps
+constexpr int kKeys = 64;                    // keys per stage (two pages)
+constexpr int kStages = 3;
+constexpr int kQTileBytes = 128 * kD * 2;    // 32 KB
+constexpr int kKVBytes = kKeys * kD * 2;     // 16 KB each for K and V
+constexpr int kPBytes = 128 * kKeys * 2;     // 16 KB per query tile
+constexpr int kMaxChunkPages = 1024;
+constexpr float kRescaleThreshold = 8.f;     // log2 units
+constexpr uint32_t kTmemCols = 512;
+// shared memory: Q (2 tiles) | stages x (K, V) | P (2 tiles)
+constexpr int kOffQ = 0;
+constexpr int kOffKV = kOffQ + 2 * kQTileBytes;
+constexpr int kOffP = kOffKV + kStages * 2 * kKVBytes;
+constexpr int kSmemBytes = kOffP + 2 * kPBytes + 1024;  // + alignment slack
+
+struct AttnTcArgs {
+  const int32_t* page_table;
+  const int32_t* n_blocks;
+  int max_blocks;
+  long long n_pages;
+  int Hq, Hkv, G, R;       // R = G * 32 query rows per CTA
+  int ppc, max_chunks;
+  int kv_rows_total;       // rows of the page-pool tensor map (OOB row for padding)
+  float* part_o;
+  float* part_ml;
+  bf16* out;
+  int32_t* status;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                   const __grid_constant__ CUtensorMap tm_blk, AttnTcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  __shared__ uint64_t q_full;
+  __shared__ uint64_t kv_full[kStages], kv_empty[kStages];
+  __shared__ uint64_t s_full[2][2], s_free[2][2];
+  __shared__ uint64_t p_full[2], p_free[2];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int pages[kMaxChunkPages];
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int c = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+  const int nb = min(max(a.n_blocks[s], 0), a.max_blocks);
+  const int total = nb + 1;  // cached pages + the current block
+  const int p0 = c * a.ppc;
+  if (p0 >= total) return;
+  const int p1 = min(total, p0 + a.ppc);
+  const int n_pg = p1 - p0;
+  const int n_tiles = (n_pg + 1) / 2;
+  const int nq = (a.R + 127) / 128;
+
+  for (int i = threadIdx.x; i < n_pg; i += blockDim.x) {
+    const int p = p0 + i;
+    int pg = -1;  // -1: the current block's page in the workspace
+    if (p < nb) {
+      pg = a.page_table[static_cast<size_t>(s) * a.max_blocks + p];
+      if (pg < 0 || pg >= a.n_pages) pg = -2;  // host-validated; read zeros if not
+    }
+    pages[i] = pg;
+  }
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&q_full, 1);
+    for (int i = 0; i < kStages; ++i) {
+      tc::mbar_init(&kv_full[i], 1);
+      tc::mbar_init(&kv_empty[i], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      for (int b = 0; b < 2; ++b) {
+        tc::mbar_init(&s_full[t][b], 1);
+        tc::mbar_init(&s_free[t][b], 4);
+      }
+      tc::mbar_init(&p_full[t], 4);
+      tc::mbar_init(&p_free[t], 1);
+    }
+    tc::fence_barrier_init();
+    tc::fence_proxy_async();
+  }
+  if (warp == 1) tc::tmem_alloc(&tmem_slot, kTmemCols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const uint32_t sbase = tc::smem_u32(smem);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_q);
+      tc::prefetch_tmap(&tm_kv);
+      tc::prefetch_tmap(&tm_blk);
+      const uint64_t pol_kv = tc::policy_evict_first();
+      const uint64_t pol_q = tc::policy_evict_last();
+      const int qrow0 = (s * a.Hq + g * a.G) * kBlock;
+      tc::mbar_arrive_expect_tx(&q_full, nq * kQTileBytes);
+      for (int t = 0; t < nq; ++t)
+        for (int dh = 0; dh < 2; ++dh)
+          tc::tma_load_2d(smem + kOffQ + t * kQTileBytes + dh * (kQTileBytes / 2), &tm_q, &q_full,
+                          dh * 64, qrow0 + 128 * t, pol_q);
+      int st = 0;
+      uint32_t ph = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        if (!tc::mbar_wait(&kv_empty[st], ph ^ 1, a.status)) break;
+        tc::mbar_arrive_expect_tx(&kv_full[st], 2 * kKVBytes);
+        uint8_t* kdst = smem + kOffKV + st * 2 * kKVBytes;
+        uint8_t* vdst = kdst + kKVBytes;
+        for (int half = 0; half < 2; ++half) {
+          const int i = 2 * j + half;
+          const CUtensorMap* m = &tm_kv;
+          int rk, rv;
+          if (i >= n_pg || pages[i] == -2) {  // padding page: rows past the end read as zeros
+            rk = rv = a.kv_rows_total;
+          } else if (pages[i] == -1) {
+            m = &tm_blk;
+            rk = ((s * 2 + 0) * a.Hkv + g) * kBlock;
+            rv = ((s * 2 + 1) * a.Hkv + g) * kBlock;
+          } else {
+            rk = ((pages[i] * 2 + 0) * a.Hkv + g) * kBlock;
+            rv = ((pages[i] * 2 + 1) * a.Hkv + g) * kBlock;
+          }
+          for (int dh = 0; dh < 2; ++dh) {
+            tc::tma_load_2d(kdst + dh * (kKVBytes / 2) + half * 4096, m, &kv_full[st], dh * 64, rk,
+                            pol_kv);
+            tc::tma_load_2d(vdst + dh * (kKVBytes / 2) + half * 4096, m, &kv_full[st], dh * 64, rv,
+                            pol_kv);
+          }
+        }
+        if (++st == kStages) { st = 0; ph ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t id_qk = tc::idesc_bf16_f32(128, kKeys);
+      const uint32_t id_pv = tc::idesc_bf16_f32_bmn(128, kD);
+      bool ok = tc::mbar_wait(&q_full, 0, a.status);
+      tc::tc_fence_after();
+      auto issue_qk = [&](int j, int st) {
+        const uint32_t kaddr = sbase + kOffKV + st * 2 * kKVBytes;
+        for (int t = 0; t < nq && ok; ++t) {
+          const int b = j & 1;
+          if (!tc::mbar_wait(&s_free[t][b], ((j >> 1) & 1) ^ 1, a.status)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t qaddr = sbase + kOffQ + t * kQTileBytes;
+          const uint32_t d = tmem + t * 128 + b * 64;
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
+            tc::mma_bf16_ss(d, tc::sdesc_kmajor_sw128(qaddr + (kk >> 2) * (kQTileBytes / 2) + off),
+                            tc::sdesc_kmajor_sw128(kaddr + (kk >> 2) * (kKVBytes / 2) + off),
+                            id_qk, kk != 0);
+          }
+          tc::mma_commit(&s_full[t][b]);
+        }
+      };
+      int st = 0;
+      uint32_t ph = 0;
+      if (ok && n_tiles > 0) {
+        ok = tc::mbar_wait(&kv_full[0], 0, a.status);
+        tc::tc_fence_after();
+        if (ok) issue_qk(0, 0);
+      }
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        int st1 = st + 1 == kStages ? 0 : st + 1;
+        uint32_t ph1 = st + 1 == kStages ? ph ^ 1 : ph;
+        if (j + 1 < n_tiles) {
+          if (!tc::mbar_wait(&kv_full[st1], ph1, a.status)) { ok = false; break; }
+          tc::tc_fence_after();
+          issue_qk(j + 1, st1);
+        }
+        const uint32_t vaddr = sbase + kOffKV + st * 2 * kKVBytes + kKVBytes;
+        for (int t = 0; t < nq && ok; ++t) {
+          if (!tc::mbar_wait(&p_full[t], j & 1, a.status)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t paddr = sbase + kOffP + t * kPBytes;
+          const uint32_t d = tmem + 256 + t * 128;
+#pragma unroll
+          for (int kk = 0; kk < kKeys / 16; ++kk)
+            tc::mma_bf16_ss(d, tc::sdesc_kmajor_sw128(paddr + kk * 32),
+                            tc::sdesc_mnmajor_sw128(vaddr + kk * 16 * 128, kKVBytes / 2), id_pv,
+                            (j | kk) != 0);
+          tc::mma_commit(&p_free[t]);
+        }
+        tc::mma_commit(&kv_empty[st]);
+        st = st1;
+        ph = ph1;
+      }
+    }
+  } else if (warp >= 4 && (warp - 4) / 4 < nq) {
+    // ------------------------------------------------ softmax / correction
+    const int t = (warp - 4) / 4;
+    const int q = warp & 3;
+    const int r = 128 * t + 32 * q + lane;  // query row of this thread
+    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+    const float scale = kLog2e * rsqrtf(static_cast<float>(kD));
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    const uint32_t prow = sbase + kOffP + t * kPBytes + (32 * q + lane) * 128;
+    const int rsw = (32 * q + lane) & 7;  // 128-byte swizzle phase of this row
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      const int b = j & 1;
+      const int valid = min(kKeys, kBlock * (n_pg - 2 * j));
+      if (!tc::mbar_wait_warp(&s_full[t][b], (j >> 1) & 1, a.status)) { ok = false; break; }
+      tc::tc_fence_after();
+      uint32_t sr[64];
+      {
+        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+        tc::tmem_ld_32x32b_x32(tmem + lane_off + t * 128 + b * 64, lo);
+        tc::tmem_ld_32x32b_x32(tmem + lane_off + t * 128 + b * 64 + 32, hi);
+      }
+      tc::tmem_ld_wait();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&s_free[t][b]);
+      float x[64];
+      float mt = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 64; ++k) {
+        x[k] = (k < valid) ? __uint_as_float(sr[k]) * scale : -INFINITY;
+        mt = fmaxf(mt, x[k]);
+      }
+      const float m_new = fmaxf(m, mt);
+      const bool rescale = (m == -INFINITY) || (m_new - m > kRescaleThreshold);
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
+        m = m_new;
+      }
+      uint32_t pk[32];
+      float rs = 0.f;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const float e0 = fast_exp2(x[2 * k] - m);
+        const float e1 = fast_exp2(x[2 * k + 1] - m);
+        rs += e0 + e1;
+        pk[k] = tc::pack_bf16x2(e0, e1);
+      }
+      l = l * alpha + rs;
+      // P buffer and O are free once the previous P V product has completed.
+      if (!tc::mbar_wait_warp(&p_free[t], (j & 1) ^ 1, a.status)) { ok = false; break; }
+      tc::tc_fence_after();
+      // The TMEM accesses are warp-collective: the warp rescales together when
+      // any of its rows needs it, the other rows with a factor of 1.
+      const bool need = rescale && j > 0;
+      if (__any_sync(0xffffffffu, need)) {
+        const float f = need ? alpha : 1.f;
+        const uint32_t o_addr = tmem + lane_off + 256 + t * 128;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t ov[32];
+          tc::tmem_ld_32x32b_x32(o_addr + cc * 32, ov);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
+          tc::tmem_st_32x32b_x32(o_addr + cc * 32, ov);
+        }
+        tc::tmem_st_wait();
+      }
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        tc::st_shared_v4(prow + ((ch ^ rsw) << 4), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2],
+                         pk[4 * ch + 3]);
+      tc::fence_proxy_async();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&p_full[t]);
+    }
+    // ---------------------------------------------------------------- output
+    // Warp-uniform: the wait verdict is shared by the warp, and R is a
+    // multiple of 32, so each warp's rows are all valid or all padding.
+    if (ok && tc::mbar_wait_warp(&p_free[t], (n_tiles - 1) & 1, a.status)) {
+      tc::tc_fence_after();
+      if (32 * (r / 32) < a.R) {
+        const int h = g * a.G + r / kBlock;
+        const int pos = r % kBlock;
+        const bool single = (total <= a.ppc) || (a.max_chunks == 1);
+        const uint32_t o_addr = tmem + lane_off + 256 + t * 128;
+        const float inv = 1.f / l;
+        bf16* dst = a.out + ((static_cast<size_t>(s) * kBlock + pos) * a.Hq + h) * kD;
+        const size_t prow_idx = ((static_cast<size_t>(s) * a.Hq + h) * a.max_chunks + c) * kBlock + pos;
+        float* po = a.part_o + prow_idx * kD;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t ov[32];
+          tc::tmem_ld_32x32b_x32(o_addr + cc * 32, ov);
+          tc::tmem_ld_wait();
+          if (single) {
+            uint32_t pkd[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              pkd[k] = tc::pack_bf16x2(__uint_as_float(ov[2 * k]) * inv,
+                                       __uint_as_float(ov[2 * k + 1]) * inv);
+            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              d4[k] = make_uint4(pkd[4 * k], pkd[4 * k + 1], pkd[4 * k + 2], pkd[4 * k + 3]);
+          } else {
+            float4* p4 = reinterpret_cast<float4*>(po + cc * 32);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              p4[k] = make_float4(__uint_as_float(ov[4 * k]), __uint_as_float(ov[4 * k + 1]),
+                                  __uint_as_float(ov[4 * k + 2]), __uint_as_float(ov[4 * k + 3]));
+          }
+        }
+        if (!single) {
+          a.part_ml[prow_idx * 2 + 0] = m;
+          a.part_ml[prow_idx * 2 + 1] = l;
+        }
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), rows};
+  const cuuint64_t strides[1] = {kD * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool attn_tc_supported(const bd_attn_shape& sh) {
+  const int G = sh.n_heads_q / sh.n_heads_kv;
+  return sh.dtype == BD_BF16 && sh.head_dim == kD && G * kBlock <= 256;
+}
+
+int attn_tc_max_chunk_pages() { return kMaxChunkPages; }
+
+cudaError_t launch_attn_tc(const bd_attn_shape& sh, const bd_kv_cache& c, int ppc, int max_chunks,
+                           const void* ws_q, const void* ws_blk, float* part_o, float* part_ml,
+                           void* out, int32_t* status, cudaStream_t st) {
+  const int B = c.batch, Hq = sh.n_heads_q, Hkv = sh.n_heads_kv;
+  CUtensorMap tm_q, tm_kv, tm_blk;
+  const uint64_t kv_rows = static_cast<uint64_t>(c.n_pages) * 2 * Hkv * kBlock;
+  if (kv_rows >= (1ull << 31)) return cudaErrorInvalidValue;
+  if (!make_tmap(&tm_q, ws_q, static_cast<uint64_t>(B) * Hq * kBlock, 128) ||
+      !make_tmap(&tm_kv, c.pages, kv_rows, kBlock) ||
+      !make_tmap(&tm_blk, ws_blk, static_cast<uint64_t>(B) * 2 * Hkv * kBlock, kBlock))
+    return cudaErrorInvalidValue;
+  AttnTcArgs a{};
+  a.page_table = c.page_table;
+  a.n_blocks = c.n_blocks;
+  a.max_blocks = c.max_blocks;
+  a.n_pages = c.n_pages;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.R = a.G * kBlock;
+  a.ppc = ppc;
+  a.max_chunks = max_chunks;
+  a.kv_rows_total = static_cast<int>(kv_rows);
+  a.part_o = part_o;
+  a.part_ml = part_ml;
+  a.out = static_cast<bf16*>(out);
+  a.status = status;
+  cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  attn_tc_kernel<<<dim3(max_chunks, Hkv, B), kThreads, kSmemBytes, st>>>(tm_q, tm_kv, tm_blk, a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace bd

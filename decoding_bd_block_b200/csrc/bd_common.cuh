@@ -106,10 +106,17 @@ cudaError_t launch_cache_commit(const bd_attn_shape& sh, const bd_kv_cache& c, c
 
 // Block attention plan: pages per split-KV chunk and the largest chunk count.
 struct AttnPlan {
+  bool tc;  // tcgen05 path (bf16, head_dim 128, G * 32 <= 256 query rows)
   int pages_per_chunk;
   int max_chunks;
-  size_t off_q, off_blk, off_o, off_ml, total;
+  size_t off_q, off_blk, off_o, off_ml, off_status, total;
 };
+// Tensor-core block attention (attn_tc.cu).
+bool attn_tc_supported(const bd_attn_shape& sh);
+int attn_tc_max_chunk_pages();
+cudaError_t launch_attn_tc(const bd_attn_shape& sh, const bd_kv_cache& c, int ppc, int max_chunks,
+                           const void* ws_q, const void* ws_blk, float* part_o, float* part_ml,
+                           void* out, int32_t* status, cudaStream_t st);
 AttnPlan plan_block_attn(const bd_attn_shape& sh, const bd_kv_cache& c);
 cudaError_t launch_block_attn(const bd_attn_shape& sh, const bd_kv_cache& c, const AttnPlan& p,
                               const void* q, const void* k, const void* v, void* out, void* ws,

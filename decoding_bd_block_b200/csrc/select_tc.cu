@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = t0, it = 0; t < t1 && ok; ++t, ++it) {
       const int b = it & 1;
       const uint32_t tph = (it >> 1) & 1;
-      if (!tc::mbar_wait(&tfull_bar[b], tph, a.status)) { ok = false; break; }
+      if (!tc::mbar_wait_warp(&tfull_bar[b], tph, a.status)) { ok = false; break; }
       tc::tc_fence_after();
       const int v = t * kVTile + q * 32 + lane;  // vocab row of this thread's lane
       const bool v_ok = v < a.V;

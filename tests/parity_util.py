@@ -24,6 +24,33 @@ def oracle_block_attn(cfg, attn_in, seqs=None):
     return res
 
 
+def _bf16_round(x):
+    """Round float64 values to bf16 (nearest even), as the kernel stores them."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    b = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def bf16_storage_block_attn(cfg, attn_in, seqs=None):
+    """The oracle's block attention with the rotated q and keys rounded to bf16,
+    i.e. the precision of the library's cache pages and rotated queries.  Used
+    to separate storage rounding from the kernel's own arithmetic error."""
+    seqs = range(cfg.batch) if seqs is None else seqs
+    res = {}
+    th = cfg.rope_theta
+    for s in seqs:
+        P = int(attn_in["prefix_len"][s])
+        kc = O.rope(O.widen(attn_in["prefix_k"][s], cfg.dtype), np.arange(P), th)
+        vc = O.widen(attn_in["prefix_v"][s], cfg.dtype)
+        pos = np.arange(P, P + 32)
+        q = _bf16_round(O.rope(O.widen(attn_in["q"][s], cfg.dtype), pos, th))
+        kb = _bf16_round(O.rope(O.widen(attn_in["k_blk"][s], cfg.dtype), pos, th))
+        keys = np.concatenate([_bf16_round(kc), kb])
+        vals = np.concatenate([vc, O.widen(attn_in["v_blk"][s], cfg.dtype)])
+        res[s] = O.attention(q, keys, vals)
+    return res
+
+
 def compare_select(ref, tokens, unmask, pmax, argmax, masked_bits):
     """Bit-exact decisions and tokens outside the ambiguity flags.
 

@@ -11,7 +11,7 @@ import pytest
 
 import oracle as O
 from decoding_bd_block_b200 import workloads as W
-from parity_util import ATOL, compare_select, oracle_block_attn
+from parity_util import ATOL, bf16_storage_block_attn, compare_select, oracle_block_attn
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -88,6 +88,12 @@ ATTN_CASES = [
                         prefix_tokens=(0,), seed=92),
     dataclasses.replace(W.QWEN7B_RAGGED, name="bf16_g7_long_ragged", batch=3,
                         prefix_range=(), prefix_tokens=(4096, 32, 2080), seed=93),
+    # one 128-row query tile (G = 4), odd page counts
+    dataclasses.replace(W.QWEN15B_STEP, name="bf16_g4_odd_pages", n_heads_q=8, n_heads_kv=2,
+                        batch=3, prefix_tokens=(0, 96, 1024), seed=101),
+    # G = 1: 32 query rows per CTA
+    dataclasses.replace(W.QWEN15B_STEP, name="bf16_g1", n_heads_q=4, n_heads_kv=4,
+                        prefix_tokens=(64,), seed=102),
 ]
 
 
@@ -112,6 +118,35 @@ def test_block_attn_longctx_sampled():
     for s, r in ref.items():
         err = float(np.abs(got[s] - r).max())
         assert err <= ATOL["bf16"], (s, err)
+
+
+def test_block_attn_growing_scores_rescale():
+    # Keys grow page by page (up to 4x), so the running max keeps rising across
+    # the KV stream and the online softmax must rescale its accumulator (about
+    # one rescale per query row).  Scores this large make the bf16 storage of
+    # the rotated q / K (the cache format) itself worth ~3e-2 against fp64, so
+    # the kernel is held to 2e-2 against the same computation with that
+    # storage rounding applied, and to that storage error + 2e-2 against the
+    # oracle.
+    from decoding_bd_block_b200.step import DecodeStep
+    cfg = dataclasses.replace(W.QWEN7B_RAGGED, name="bf16_growing", batch=2, prefix_range=(),
+                              prefix_tokens=(3072, 1504), seed=103)
+    a = W.make_attn_inputs(cfg)
+    for s in range(cfg.batch):
+        k = W.f32_from_bf16_bits(a["prefix_k"][s])
+        ramp = (1.0 + np.arange(k.shape[0]) / 1024.0).astype(np.float32)[:, None, None]
+        a["prefix_k"][s] = W.bf16_bits_from_f32(k * ramp)
+    a["k_blk"] = W.bf16_bits_from_f32(W.f32_from_bf16_bits(a["k_blk"]) * 4.0)
+    step = DecodeStep(cfg, a, None)
+    step.run_attn()
+    torch.cuda.synchronize()
+    got = step.out.float().cpu().numpy()
+    ref = oracle_block_attn(cfg, a)
+    emu = bf16_storage_block_attn(cfg, a)
+    for s in ref:
+        storage = float(np.abs(emu[s] - ref[s]).max())
+        assert float(np.abs(got[s] - emu[s]).max()) <= ATOL["bf16"]
+        assert float(np.abs(got[s] - ref[s]).max()) <= storage + ATOL["bf16"]
 
 
 def test_block_attn_repeatable_and_after_commit():
