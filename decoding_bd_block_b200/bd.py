@@ -22,7 +22,8 @@ STATUS = {0: "BD_OK", -1: "BD_ERR_INVALID_ARG", -2: "BD_ERR_UNSUPPORTED",
 EXPORTED = ("bd_cache_commit", "bd_block_attn_workspace_size", "bd_block_attn",
             "bd_confidence_select_workspace_size", "bd_confidence_select",
             "bd_block_mask_attn", "bd_status_string", "bd_last_cuda_error_string",
-            "bd_kernel_launches")
+            "bd_kernel_launches", "bd_confidence_select_noalloc")
+BD_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 if not os.path.exists(_LIB_PATH):
     raise ImportError(f"libbd.so not built ({_LIB_PATH}); run "
@@ -66,6 +67,8 @@ _SIGS = {
     "bd_confidence_select": [_I, _I, _I, _I, _P, _P, _P, _P, ctypes.c_float, _I, _P, _P, _P, _P,
                              _P, ctypes.c_size_t, _P],
     "bd_block_mask_attn": [ctypes.POINTER(bd_attn_shape), _P, _P, _P, _P, _I, _I, _I, _P],
+    "bd_confidence_select_noalloc": [_I, _I, _I, _I, _P, _P, _P, _P, ctypes.c_float, _I, _P, _P,
+                                     _P, _P, _P],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -181,6 +184,17 @@ def bd_confidence_select(dtype, batch, hidden, vocab, h, h_prev, w_lm, masked_bi
         _ptr(w_lm), _ptr(masked_bits), float(tau), int(sub_block), _ptr(tokens),
         _ptr(unmask_bits), _ptr(pmax_out), _ptr(argmax_out), _ptr(workspace), int(wsb),
         _stream(stream)))
+
+
+def bd_confidence_select_noalloc(dtype, batch, hidden, vocab, h, h_prev, w_lm, masked_bits, tau,
+                                 sub_block, tokens, unmask_bits, pmax_out, argmax_out,
+                                 stream=None):
+    """bd_confidence_select for callers that cannot allocate a workspace: the
+    library's own fixed device scratch is used instead (see include/bd.h)."""
+    _check("bd_confidence_select_noalloc", _lib.bd_confidence_select_noalloc(
+        dtype_code(dtype), int(batch), int(hidden), int(vocab), _ptr(h), _ptr(h_prev),
+        _ptr(w_lm), _ptr(masked_bits), float(tau), int(sub_block), _ptr(tokens),
+        _ptr(unmask_bits), _ptr(pmax_out), _ptr(argmax_out), _stream(stream)))
 
 
 def bd_block_mask_attn(shape: bd_attn_shape, q, k, v, out, n_seqs, L, block, stream=None):

@@ -52,6 +52,10 @@ int check_cache(const bd_attn_shape* sh, const bd_kv_cache* c) {
 
 }  // namespace
 
+namespace bd {
+int report_cuda_error(cudaError_t e) { return cuda_status(e); }
+}  // namespace bd
+
 extern "C" {
 
 const char* bd_status_string(int status) {

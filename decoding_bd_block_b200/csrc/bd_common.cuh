@@ -83,6 +83,9 @@ __device__ __forceinline__ Stat stat_combine(Stat x, Stat y) {
 
 // Process-wide count of kernels enqueued by the library (bd_kernel_launches).
 void count_launches(int n);
+// Records a CUDA error for bd_last_cuda_error_string(); returns BD_ERR_CUDA
+// (BD_OK for cudaSuccess).
+int report_cuda_error(cudaError_t e);
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

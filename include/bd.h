@@ -175,6 +175,39 @@ BD_API int bd_confidence_select(int32_t dtype, int32_t batch, int32_t hidden,
                          int32_t* argmax_out, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* bd_confidence_select_noalloc -- bd_confidence_select without a workspace.
+ *
+ * The method's description has no counterpart to this call: it exists for
+ * callers that cannot allocate device memory when they run the step, such
+ * as a plugin that its host application hands only input and output
+ * buffers, code running while a framework's caching allocator owns the whole
+ * device, or a latency-bound loop that must not pay cudaMalloc's implicit
+ * device synchronisation.
+ *
+ * Same arguments, results and errors as bd_confidence_select, minus the
+ * workspace: the step's scratch lives in one fixed array of
+ * BD_NOALLOC_SCRATCH_BYTES that the library keeps in device memory on every
+ * GPU where it is loaded, until the process exits.  A step whose scratch
+ * would exceed it (roughly batch * 32 rows * hidden elements plus 12 bytes
+ * per row and SM) is refused with BD_ERR_WORKSPACE before anything runs: in
+ * bf16 on a 148-SM B200 that is a batch above 24 at hidden 3584, above 48
+ * at hidden 1536.  The call
+ * allocates nothing.  Its first call on a device looks the array's device
+ * address up (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture on the device.  Every call on a
+ * device shares the one array and leaves its contents behind for the next
+ * (nothing in it has to start at zero: each call writes every part it
+ * reads), so calls whose work overlaps on the GPU -- different streams, or
+ * different host threads on one device -- race and must be serialised by the
+ * caller. */
+#define BD_NOALLOC_SCRATCH_BYTES (8u << 20)
+BD_API int bd_confidence_select_noalloc(int32_t dtype, int32_t batch, int32_t hidden,
+                                        int32_t vocab, const void* h, const void* h_prev,
+                                        const void* w_lm, const uint32_t* masked_bits,
+                                        float tau, int32_t sub_block, int32_t* tokens,
+                                        uint32_t* unmask_bits, float* pmax_out,
+                                        int32_t* argmax_out, void* stream);
+
 /* bd_block_mask_attn -- attention of the training forward under the 2L x 2L
  * complementary mask ([N1] key design 2).
  *
