@@ -10,13 +10,18 @@
 // The chunk's pages stream through a ring of 64-key K/V stages (two pages
 // per stage, TMA with the 128-byte swizzle).  Per stage j and tile t:
 //
-//   warp 1 (one thread)  S_t = Q_t K_j^T   -> TMEM (two 64-column buffers)
-//                        O_t += P_t V_j    (P from shared memory, O in TMEM)
+//   warp 1 (one thread)  S_t = Q_t K_j^T   -> TMEM, two 64-column buffers
+//                        O_t += P_t V_j    (P read from TMEM, O in TMEM)
 //   warps 4+4t .. 7+4t   one thread per query row: online softmax in base 2
-//                        (scores pre-scaled by log2(e)/sqrt(d)), P -> bf16
-//                        into shared memory, lazy rescale of its O row in
-//                        TMEM when the running max grows by more than 2^8
+//                        (scores scaled by log2(e)/sqrt(d) inside one FMA),
+//                        P as bf16 written over its S buffer in TMEM, lazy
+//                        rescale of its O row when the running max grows by
+//                        more than 2^8
 //   warp 0 (one thread)  TMA producer: Q once, then K/V pages
+//
+// Ordering: the MMA thread reuses S buffer b for stage j+2 only after P V of
+// stage j (which reads P from that buffer) has completed; the softmax stores
+// P of stage j (and rescales O) only after P V of stage j-1 has completed.
 //
 // The chunk's (m, l, O) go to the workspace for attn_merge_kernel, or --
 // when one chunk covers the whole sequence -- O / l straight to the output.
@@ -29,18 +34,17 @@ namespace {
 constexpr int kD = 128;
 constexpr int kThreads = 384;               // 12 warps
 constexpr int kKeys = 64;                    // keys per stage (two pages)
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kQTileBytes = 128 * kD * 2;    // 32 KB
 constexpr int kKVBytes = kKeys * kD * 2;     // 16 KB each for K and V
-constexpr int kPBytes = 128 * kKeys * 2;     // 16 KB per query tile
 constexpr int kMaxChunkPages = 1024;
 constexpr float kRescaleThreshold = 8.f;     // log2 units
 constexpr uint32_t kTmemCols = 512;
-// shared memory: Q (2 tiles) | stages x (K, V) | P (2 tiles)
+// TMEM columns: S/P buffers at t * 128 + b * 64, O_t at 256 + t * 128.
+// shared memory: Q (2 tiles) | stages x (K, V)
 constexpr int kOffQ = 0;
 constexpr int kOffKV = kOffQ + 2 * kQTileBytes;
-constexpr int kOffP = kOffKV + kStages * 2 * kKVBytes;
-constexpr int kSmemBytes = kOffP + 2 * kPBytes + 1024;  // + alignment slack
+constexpr int kSmemBytes = kOffKV + kStages * 2 * kKVBytes + 1024;  // + alignment slack
 
 struct AttnTcArgs {
   const int32_t* page_table;
@@ -64,8 +68,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   __shared__ uint64_t q_full;
   __shared__ uint64_t kv_full[kStages], kv_empty[kStages];
-  __shared__ uint64_t s_full[2][2], s_free[2][2];
-  __shared__ uint64_t p_full[2], p_free[2];
+  __shared__ uint64_t s_full[2][2];
+  __shared__ uint64_t p_full[2], pv_done[2];
   __shared__ uint32_t tmem_slot;
   __shared__ int pages[kMaxChunkPages];
 
@@ -96,12 +100,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&kv_empty[i], 1);
     }
     for (int t = 0; t < 2; ++t) {
-      for (int b = 0; b < 2; ++b) {
-        tc::mbar_init(&s_full[t][b], 1);
-        tc::mbar_init(&s_free[t][b], 4);
-      }
+      for (int b = 0; b < 2; ++b) tc::mbar_init(&s_full[t][b], 1);
       tc::mbar_init(&p_full[t], 4);
-      tc::mbar_init(&p_free[t], 1);
+      tc::mbar_init(&pv_done[t], 1);
     }
     tc::fence_barrier_init();
     tc::fence_proxy_async();
@@ -165,11 +166,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id_pv = tc::idesc_bf16_f32_bmn(128, kD);
       bool ok = tc::mbar_wait(&q_full, 0, a.status);
       tc::tc_fence_after();
+      // S_t(j) = Q_t K_j^T into buffer j & 1.  The buffer last held P_t(j-2):
+      // wait until P V of stage j-2 has completed before overwriting it.
       auto issue_qk = [&](int j, int st) {
         const uint32_t kaddr = sbase + kOffKV + st * 2 * kKVBytes;
         for (int t = 0; t < nq && ok; ++t) {
           const int b = j & 1;
-          if (!tc::mbar_wait(&s_free[t][b], ((j >> 1) & 1) ^ 1, a.status)) { ok = false; break; }
+          if (j >= 2 && !tc::mbar_wait(&pv_done[t], (j - 2) & 1, a.status)) { ok = false; break; }
           tc::tc_fence_after();
           const uint32_t qaddr = sbase + kOffQ + t * kQTileBytes;
           const uint32_t d = tmem + t * 128 + b * 64;
@@ -202,14 +205,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < nq && ok; ++t) {
           if (!tc::mbar_wait(&p_full[t], j & 1, a.status)) { ok = false; break; }
           tc::tc_fence_after();
-          const uint32_t paddr = sbase + kOffP + t * kPBytes;
+          const uint32_t pbuf = tmem + t * 128 + (j & 1) * 64;  // P_t(j), 32 packed columns
           const uint32_t d = tmem + 256 + t * 128;
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk)
-            tc::mma_bf16_ss(d, tc::sdesc_kmajor_sw128(paddr + kk * 32),
+            tc::mma_bf16_ts(d, pbuf + kk * 8,
                             tc::sdesc_mnmajor_sw128(vaddr + kk * 16 * 128, kKVBytes / 2), id_pv,
                             (j | kk) != 0);
-          tc::mma_commit(&p_free[t]);
+          tc::mma_commit(&pv_done[t]);
         }
         tc::mma_commit(&kv_empty[st]);
         st = st1;
@@ -225,31 +228,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float scale = kLog2e * rsqrtf(static_cast<float>(kD));
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    const uint32_t prow = sbase + kOffP + t * kPBytes + (32 * q + lane) * 128;
-    const int rsw = (32 * q + lane) & 7;  // 128-byte swizzle phase of this row
     for (int j = 0; j < n_tiles && ok; ++j) {
       const int b = j & 1;
       const int valid = min(kKeys, kBlock * (n_pg - 2 * j));
       if (!tc::mbar_wait_warp(&s_full[t][b], (j >> 1) & 1, a.status)) { ok = false; break; }
       tc::tc_fence_after();
+      const uint32_t sbuf = tmem + lane_off + t * 128 + b * 64;
       uint32_t sr[64];
       {
         uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
         uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        tc::tmem_ld_32x32b_x32(tmem + lane_off + t * 128 + b * 64, lo);
-        tc::tmem_ld_32x32b_x32(tmem + lane_off + t * 128 + b * 64 + 32, hi);
+        tc::tmem_ld_32x32b_x32(sbuf, lo);
+        tc::tmem_ld_32x32b_x32(sbuf + 32, hi);
       }
       tc::tmem_ld_wait();
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&s_free[t][b]);
-      float x[64];
-      float mt = -INFINITY;
+      if (valid < kKeys) {  // warp-uniform: only the last stage of a chunk can be half full
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        x[k] = (k < valid) ? __uint_as_float(sr[k]) * scale : -INFINITY;
-        mt = fmaxf(mt, x[k]);
+        for (int k = 32; k < 64; ++k) sr[k] = __float_as_uint(-INFINITY);
       }
+      float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int k = 0; k < 64; ++k) mk[k & 3] = fmaxf(mk[k & 3], __uint_as_float(sr[k]));
+      const float mt = fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])) * scale;
       const float m_new = fmaxf(m, mt);
       const bool rescale = (m == -INFINITY) || (m_new - m > kRescaleThreshold);
       float alpha = 1.f;
@@ -257,20 +257,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
         m = m_new;
       }
+      const float neg_m = -m;
       uint32_t pk[32];
-      float rs = 0.f;
+      float rk[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
-        const float e0 = fast_exp2(x[2 * k] - m);
-        const float e1 = fast_exp2(x[2 * k + 1] - m);
-        rs += e0 + e1;
+        const float e0 = fast_exp2(fmaf(__uint_as_float(sr[2 * k]), scale, neg_m));
+        const float e1 = fast_exp2(fmaf(__uint_as_float(sr[2 * k + 1]), scale, neg_m));
+        rk[k & 3] += e0 + e1;
         pk[k] = tc::pack_bf16x2(e0, e1);
       }
-      l = l * alpha + rs;
-      // P buffer and O are free once the previous P V product has completed.
-      if (!tc::mbar_wait_warp(&p_free[t], (j & 1) ^ 1, a.status)) { ok = false; break; }
-      tc::tc_fence_after();
-      // The TMEM accesses are warp-collective: the warp rescales together when
+      l = l * alpha + ((rk[0] + rk[1]) + (rk[2] + rk[3]));
+      // No tensor-memory store while the previous P V product (a TS MMA that
+      // reads P from tensor memory) may still run: on B200 a store into
+      // another column range during that product corrupted results in
+      // testing.  The wait also makes O stable for the rescale below.
+      if (j > 0) {
+        if (!tc::mbar_wait_warp(&pv_done[t], (j - 1) & 1, a.status)) { ok = false; break; }
+        tc::tc_fence_after();
+      }
+      // TMEM accesses are warp-collective, so the warp rescales together when
       // any of its rows needs it, the other rows with a factor of 1.
       const bool need = rescale && j > 0;
       if (__any_sync(0xffffffffu, need)) {
@@ -285,13 +291,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
           tc::tmem_st_32x32b_x32(o_addr + cc * 32, ov);
         }
-        tc::tmem_st_wait();
       }
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        tc::st_shared_v4(prow + ((ch ^ rsw) << 4), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2],
-                         pk[4 * ch + 3]);
-      tc::fence_proxy_async();
+      // P over the first 32 columns of this S buffer (two bf16 per column).
+      tc::tmem_st_32x32b_x32(sbuf, pk);
+      tc::tmem_st_wait();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&p_full[t]);
@@ -299,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- output
     // Warp-uniform: the wait verdict is shared by the warp, and R is a
     // multiple of 32, so each warp's rows are all valid or all padding.
-    if (ok && tc::mbar_wait_warp(&p_free[t], (n_tiles - 1) & 1, a.status)) {
+    if (ok && tc::mbar_wait_warp(&pv_done[t], (n_tiles - 1) & 1, a.status)) {
       tc::tc_fence_after();
       if (32 * (r / 32) < a.R) {
         const int h = g * a.G + r / kBlock;

@@ -33,7 +33,7 @@ constexpr int kMaxN = 256;         // packed rows per group (MMA N)
 constexpr int kMaxStages = 12;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kWBytes = kVTile * kKStage * 2;  // 16 KB
-constexpr int kSmemBytes = 200 * 1024;  // + ~12.5 KB static stays under 227 KB
+constexpr int kSmemBytes = 192 * 1024;  // + ~29 KB static stays under 227 KB
 
 struct SelectTcArgs {
   const int32_t* count;  // M (written by the gather kernel)
@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ float red_m[4][kMaxN];
   __shared__ float red_s[4][kMaxN];
   __shared__ int red_a[4][kMaxN];
+  __shared__ float xpose[4][32 * 33];  // per epilogue warp: a 32 x 32 chunk, transposed
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int M = *a.count;
@@ -170,9 +171,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tph = (it >> 1) & 1;
       if (!tc::mbar_wait_warp(&tfull_bar[b], tph, a.status)) { ok = false; break; }
       tc::tc_fence_after();
-      const int v = t * kVTile + q * 32 + lane;  // vocab row of this thread's lane
-      const bool v_ok = v < a.V;
-      const int vbase = t * kVTile + q * 32;
+      const int vbase = t * kVTile + q * 32;  // vocab row of this warp's lane 0
+      // Each 32-lane x 32-column chunk goes through shared memory transposed,
+      // so that thread `lane` folds column (c * 32 + lane) -- one packed row
+      // -- over this warp's 32 vocab rows with plain per-thread arithmetic.
+      const bool full_tile = vbase + 32 <= a.V;
+      float* tb = xpose[q];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         if (c < n_chunks) {
@@ -181,29 +185,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  r);
           tc::tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float x = v_ok ? __uint_as_float(r[j]) : -INFINITY;
-            const float mx = tc::redux_max_f32(x);
-            if (mx == -INFINITY) continue;  // warp-uniform
-            const uint32_t bal = __ballot_sync(0xffffffffu, x == mx);
-            const int arg = vbase + __ffs(bal) - 1;
-            float e = fast_exp2((x - mx) * kLog2e);
-            e += __shfl_xor_sync(0xffffffffu, e, 16);
-            e += __shfl_xor_sync(0xffffffffu, e, 8);
-            e += __shfl_xor_sync(0xffffffffu, e, 4);
-            e += __shfl_xor_sync(0xffffffffu, e, 2);
-            e += __shfl_xor_sync(0xffffffffu, e, 1);
-            if (lane == j) {
-              if (mx > run_m[c]) {
-                run_s[c] = run_s[c] * fast_exp2((run_m[c] - mx) * kLog2e) + e;
-                run_m[c] = mx;
-                run_a[c] = arg;
-              } else {
-                run_s[c] += e * fast_exp2((mx - run_m[c]) * kLog2e);
-                if (mx == run_m[c] && arg < run_a[c]) run_a[c] = arg;
-              }
+          for (int j = 0; j < 32; ++j) tb[j * 33 + lane] = __uint_as_float(r[j]);
+          __syncwarp();
+          const float* col = tb + lane * 33;
+          float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          int ak[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x = (full_tile || vbase + i < a.V) ? col[i] : -INFINITY;
+            if (x > mk[i & 3]) {
+              mk[i & 3] = x;
+              ak[i & 3] = i;
             }
           }
+          float mx = fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3]));
+          int am = 32;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) am = (mk[k] == mx && ak[k] < am) ? ak[k] : am;
+          if (mx != -INFINITY) {
+            const float mls = mx * kLog2e;
+            float sk[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float x = (full_tile || vbase + i < a.V) ? col[i] : -INFINITY;
+              sk[i & 3] += fast_exp2(fmaf(x, kLog2e, -mls));
+            }
+            const float e = (sk[0] + sk[1]) + (sk[2] + sk[3]);
+            const int arg = vbase + am;
+            if (mx > run_m[c]) {
+              run_s[c] = run_s[c] * fast_exp2((run_m[c] - mx) * kLog2e) + e;
+              run_m[c] = mx;
+              run_a[c] = arg;
+            } else {
+              run_s[c] += e * fast_exp2((mx - run_m[c]) * kLog2e);
+              if (mx == run_m[c] && arg < run_a[c]) run_a[c] = arg;
+            }
+          }
+          __syncwarp();
         }
       }
       tc::tc_fence_before();
