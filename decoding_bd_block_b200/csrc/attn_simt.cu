@@ -192,8 +192,8 @@ __global__ void __launch_bounds__(D) attn_merge_kernel(const int32_t* __restrict
 }
 
 // -------------------------------------------------------------- host side
-// Tensor-core split: one CTA per SM at a time, so pick the (even) chunk size
-// that minimises waves x (pages per chunk + a fixed cost) over all (chunk, kv
+// Tensor-core split: one CTA per SM at a time, so pick the chunk size (a
+// multiple of 4 pages) that minimises waves x (pages per chunk + a fixed cost) over all (chunk, kv
 // head, sequence) CTAs.  The fixed cost, worth ~8 pages of K/V traffic,
 // stands for the CTA's query load (up to 64 KB), set-up and its fp32 partial
 // (m, l, O) for the merge; at least 4 pages (two 64-key stages) per chunk.
@@ -205,7 +205,7 @@ static int plan_tc_chunk(const bd_attn_shape& sh, const bd_kv_cache& c, int max_
   const int cap = attn_tc_max_chunk_pages();
   long long best_cost = -1;
   int best = cap;
-  for (int ppc = 4; ppc <= cap; ppc += 2) {
+  for (int ppc = 4; ppc <= cap; ppc += 4) {  // whole 128-key stages
     long long ctas = 0;
     for (int s = 0; s < c.batch; ++s) ctas += (c.n_blocks_host[s] + 1 + ppc - 1) / ppc;
     ctas *= sh.n_heads_kv;

@@ -6,22 +6,28 @@
 //
 // CTA = (split-KV chunk, KV head g, sequence s).  Its query rows are the
 // G = Hq/Hkv heads of group g times the block's 32 positions (row r = head
-// (r / 32) of the group, position r % 32), one or two 128-row tiles Q_t.
-// The chunk's pages stream through a ring of 64-key K/V stages (two pages
-// per stage, TMA with the 128-byte swizzle).  Per stage j and tile t:
+// (r / 32) of the group, position r % 32), one or two 128-row tiles Q_t,
+// loaded once by TMA into shared memory.  The chunk's pages stream through
+// two 128-key K/V stages (four pages per stage, TMA, 128-byte swizzle).
 //
-//   warp 1 (one thread)  S_t = Q_t K_j^T   -> TMEM, two 64-column buffers
-//                        O_t += P_t V_j    (P read from TMEM, O in TMEM)
+// Tensor memory (512 columns): S_t at 128 t (fp32; P_t is written over its
+// first 64 columns as packed bf16), O_t at 256 + 128 t (fp32).
+//
+//   warp 1 (one thread)  ping-pong over the query tiles, per stage j:
+//                        O_t += P_t(j) V_j (TS MMA, P from TMEM), then
+//                        S_t(j+1) = Q_t K_{j+1}^T (SS MMA, N = 128 keys).
+//                        MMAs of one thread execute in issue order, so
+//                        S_t(j+1) overwrites P_t(j) only after P V has read
+//                        it, and while tile t's softmax works the tensor core
+//                        runs the other tile's products.
 //   warps 4+4t .. 7+4t   one thread per query row: online softmax in base 2
 //                        (scores scaled by log2(e)/sqrt(d) inside one FMA),
-//                        P as bf16 written over its S buffer in TMEM, lazy
-//                        rescale of its O row when the running max grows by
-//                        more than 2^8
-//   warp 0 (one thread)  TMA producer: Q once, then K/V pages
-//
-// Ordering: the MMA thread reuses S buffer b for stage j+2 only after P V of
-// stage j (which reads P from that buffer) has completed; the softmax stores
-// P of stage j (and rescales O) only after P V of stage j-1 has completed.
+//                        P as bf16 over S_t, lazy rescale of its O row when
+//                        the running max grows by more than 2^8.  Tile t's
+//                        tensor-memory stores happen only when none of tile
+//                        t's own products is in flight.
+//   warp 0               TMA producer: Q, then the K/V pages (16 lanes issue
+//                        the 16 boxes of a stage).
 //
 // The chunk's (m, l, O) go to the workspace for attn_merge_kernel, or --
 // when one chunk covers the whole sequence -- O / l straight to the output.
@@ -33,17 +39,16 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kThreads = 384;               // 12 warps
-constexpr int kKeys = 64;                    // keys per stage (two pages)
-constexpr int kStages = 4;
+constexpr int kKeys = 128;                   // keys per stage (four pages)
+constexpr int kStages = 2;
 constexpr int kQTileBytes = 128 * kD * 2;    // 32 KB
-constexpr int kKVBytes = kKeys * kD * 2;     // 16 KB each for K and V
+constexpr int kKVBytes = kKeys * kD * 2;     // 32 KB each for K and V
 constexpr int kMaxChunkPages = 1024;
 constexpr float kRescaleThreshold = 8.f;     // log2 units
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: S/P buffers at t * 128 + b * 64, O_t at 256 + t * 128.
-// shared memory: Q (2 tiles) | stages x (K, V)
+constexpr uint32_t kColS = 0, kColO = 256;
 constexpr int kOffQ = 0;
-constexpr int kOffKV = kOffQ + 2 * kQTileBytes;
+constexpr int kOffKV = 2 * kQTileBytes;
 constexpr int kSmemBytes = kOffKV + kStages * 2 * kKVBytes + 1024;  // + alignment slack
 
 struct AttnTcArgs {
@@ -68,8 +73,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   __shared__ uint64_t q_full;
   __shared__ uint64_t kv_full[kStages], kv_empty[kStages];
-  __shared__ uint64_t s_full[2][2];
-  __shared__ uint64_t p_full[2], pv_done[2];
+  __shared__ uint64_t s_full[2], p_full[2], pv_done[2];
   __shared__ uint32_t tmem_slot;
   __shared__ int pages[kMaxChunkPages];
 
@@ -81,7 +85,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (p0 >= total) return;
   const int p1 = min(total, p0 + a.ppc);
   const int n_pg = p1 - p0;
-  const int n_tiles = (n_pg + 1) / 2;
+  const int n_tiles = (n_pg + 3) / 4;
   const int nq = (a.R + 127) / 128;
 
   for (int i = threadIdx.x; i < n_pg; i += blockDim.x) {
@@ -100,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&kv_empty[i], 1);
     }
     for (int t = 0; t < 2; ++t) {
-      for (int b = 0; b < 2; ++b) tc::mbar_init(&s_full[t][b], 1);
+      tc::mbar_init(&s_full[t], 1);
       tc::mbar_init(&p_full[t], 4);
       tc::mbar_init(&pv_done[t], 1);
     }
@@ -116,103 +120,90 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------- producer
+    // The whole warp: lane 0 arms the stage's barrier, then lanes 0..15 each
+    // issue one of its sixteen 4 KB boxes (page, K or V, d half).
     if (lane == 0) {
       tc::prefetch_tmap(&tm_q);
       tc::prefetch_tmap(&tm_kv);
       tc::prefetch_tmap(&tm_blk);
-      const uint64_t pol_kv = tc::policy_evict_first();
-      const uint64_t pol_q = tc::policy_evict_last();
+    }
+    const uint64_t pol_kv = tc::policy_evict_first();
+    const uint64_t pol_q = tc::policy_evict_last();
+    if (lane == 0) {
       const int qrow0 = (s * a.Hq + g * a.G) * kBlock;
       tc::mbar_arrive_expect_tx(&q_full, nq * kQTileBytes);
       for (int t = 0; t < nq; ++t)
         for (int dh = 0; dh < 2; ++dh)
           tc::tma_load_2d(smem + kOffQ + t * kQTileBytes + dh * (kQTileBytes / 2), &tm_q, &q_full,
                           dh * 64, qrow0 + 128 * t, pol_q);
-      int st = 0;
-      uint32_t ph = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        if (!tc::mbar_wait(&kv_empty[st], ph ^ 1, a.status)) break;
-        tc::mbar_arrive_expect_tx(&kv_full[st], 2 * kKVBytes);
-        uint8_t* kdst = smem + kOffKV + st * 2 * kKVBytes;
-        uint8_t* vdst = kdst + kKVBytes;
-        for (int half = 0; half < 2; ++half) {
-          const int i = 2 * j + half;
-          const CUtensorMap* m = &tm_kv;
-          int rk, rv;
-          if (i >= n_pg || pages[i] == -2) {  // padding page: rows past the end read as zeros
-            rk = rv = a.kv_rows_total;
-          } else if (pages[i] == -1) {
-            m = &tm_blk;
-            rk = ((s * 2 + 0) * a.Hkv + g) * kBlock;
-            rv = ((s * 2 + 1) * a.Hkv + g) * kBlock;
-          } else {
-            rk = ((pages[i] * 2 + 0) * a.Hkv + g) * kBlock;
-            rv = ((pages[i] * 2 + 1) * a.Hkv + g) * kBlock;
-          }
-          for (int dh = 0; dh < 2; ++dh) {
-            tc::tma_load_2d(kdst + dh * (kKVBytes / 2) + half * 4096, m, &kv_full[st], dh * 64, rk,
-                            pol_kv);
-            tc::tma_load_2d(vdst + dh * (kKVBytes / 2) + half * 4096, m, &kv_full[st], dh * 64, rv,
-                            pol_kv);
-          }
+    }
+    const int pg = (lane >> 2) & 3, kv = (lane >> 1) & 1, dh = lane & 1;
+    int st = 0;
+    uint32_t ph = 0;
+    for (int j = 0; j < n_tiles; ++j) {
+      if (!tc::mbar_wait_warp(&kv_empty[st], ph ^ 1, a.status)) break;
+      if (lane == 0) tc::mbar_arrive_expect_tx(&kv_full[st], 2 * kKVBytes);
+      __syncwarp();
+      if (lane < 16) {
+        const int i = 4 * j + pg;
+        const CUtensorMap* m = &tm_kv;
+        int row;
+        if (i >= n_pg || pages[i] == -2) {  // padding page: rows past the end read as zeros
+          row = a.kv_rows_total;
+        } else if (pages[i] == -1) {
+          m = &tm_blk;
+          row = ((s * 2 + kv) * a.Hkv + g) * kBlock;
+        } else {
+          row = ((pages[i] * 2 + kv) * a.Hkv + g) * kBlock;
         }
-        if (++st == kStages) { st = 0; ph ^= 1; }
+        tc::tma_load_2d(smem + kOffKV + st * 2 * kKVBytes + kv * kKVBytes + dh * (kKVBytes / 2) +
+                            pg * 4096,
+                        m, &kv_full[st], dh * 64, row, pol_kv);
       }
+      if (++st == kStages) { st = 0; ph ^= 1; }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_qk = tc::idesc_bf16_f32(128, kKeys);
       const uint32_t id_pv = tc::idesc_bf16_f32_bmn(128, kD);
-      bool ok = tc::mbar_wait(&q_full, 0, a.status);
-      tc::tc_fence_after();
-      // S_t(j) = Q_t K_j^T into buffer j & 1.  The buffer last held P_t(j-2):
-      // wait until P V of stage j-2 has completed before overwriting it.
-      auto issue_qk = [&](int j, int st) {
+      auto issue_qk = [&](int t, int st) {  // S_t = Q_t K^T, K = d: 8 steps of 16
+        const uint32_t qaddr = sbase + kOffQ + t * kQTileBytes;
         const uint32_t kaddr = sbase + kOffKV + st * 2 * kKVBytes;
-        for (int t = 0; t < nq && ok; ++t) {
-          const int b = j & 1;
-          if (j >= 2 && !tc::mbar_wait(&pv_done[t], (j - 2) & 1, a.status)) { ok = false; break; }
-          tc::tc_fence_after();
-          const uint32_t qaddr = sbase + kOffQ + t * kQTileBytes;
-          const uint32_t d = tmem + t * 128 + b * 64;
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
-            tc::mma_bf16_ss(d, tc::sdesc_kmajor_sw128(qaddr + (kk >> 2) * (kQTileBytes / 2) + off),
-                            tc::sdesc_kmajor_sw128(kaddr + (kk >> 2) * (kKVBytes / 2) + off),
-                            id_qk, kk != 0);
-          }
-          tc::mma_commit(&s_full[t][b]);
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32;
+          tc::mma_bf16_ss(tmem + kColS + t * 128,
+                          tc::sdesc_kmajor_sw128(qaddr + (kk >> 2) * (kQTileBytes / 2) + off),
+                          tc::sdesc_kmajor_sw128(kaddr + (kk >> 2) * (kKVBytes / 2) + off), id_qk,
+                          kk != 0);
         }
+        tc::mma_commit(&s_full[t]);
       };
+      bool ok = tc::mbar_wait(&q_full, 0, a.status) && tc::mbar_wait(&kv_full[0], 0, a.status);
+      tc::tc_fence_after();
+      for (int t = 0; t < nq && ok; ++t) issue_qk(t, 0);
       int st = 0;
       uint32_t ph = 0;
-      if (ok && n_tiles > 0) {
-        ok = tc::mbar_wait(&kv_full[0], 0, a.status);
-        tc::tc_fence_after();
-        if (ok) issue_qk(0, 0);
-      }
       for (int j = 0; j < n_tiles && ok; ++j) {
-        int st1 = st + 1 == kStages ? 0 : st + 1;
-        uint32_t ph1 = st + 1 == kStages ? ph ^ 1 : ph;
-        if (j + 1 < n_tiles) {
-          if (!tc::mbar_wait(&kv_full[st1], ph1, a.status)) { ok = false; break; }
-          tc::tc_fence_after();
-          issue_qk(j + 1, st1);
-        }
+        const int st1 = st + 1 == kStages ? 0 : st + 1;
+        const uint32_t ph1 = st + 1 == kStages ? ph ^ 1 : ph;
+        const bool more = j + 1 < n_tiles;
         const uint32_t vaddr = sbase + kOffKV + st * 2 * kKVBytes + kKVBytes;
         for (int t = 0; t < nq && ok; ++t) {
           if (!tc::mbar_wait(&p_full[t], j & 1, a.status)) { ok = false; break; }
           tc::tc_fence_after();
-          const uint32_t pbuf = tmem + t * 128 + (j & 1) * 64;  // P_t(j), 32 packed columns
-          const uint32_t d = tmem + 256 + t * 128;
 #pragma unroll
-          for (int kk = 0; kk < kKeys / 16; ++kk)
-            tc::mma_bf16_ts(d, pbuf + kk * 8,
+          for (int kk = 0; kk < kKeys / 16; ++kk)  // O_t += P_t V_j, K = keys: 8 steps of 16
+            tc::mma_bf16_ts(tmem + kColO + t * 128, tmem + kColS + t * 128 + kk * 8,
                             tc::sdesc_mnmajor_sw128(vaddr + kk * 16 * 128, kKVBytes / 2), id_pv,
                             (j | kk) != 0);
           tc::mma_commit(&pv_done[t]);
+          if (more) {
+            if (t == 0 && !tc::mbar_wait(&kv_full[st1], ph1, a.status)) { ok = false; break; }
+            tc::tc_fence_after();
+            issue_qk(t, st1);
+          }
         }
         tc::mma_commit(&kv_empty[st]);
         st = st1;
@@ -228,27 +219,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float scale = kLog2e * rsqrtf(static_cast<float>(kD));
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    const uint32_t sbuf = tmem + lane_off + kColS + t * 128;
     for (int j = 0; j < n_tiles && ok; ++j) {
-      const int b = j & 1;
-      const int valid = min(kKeys, kBlock * (n_pg - 2 * j));
-      if (!tc::mbar_wait_warp(&s_full[t][b], (j >> 1) & 1, a.status)) { ok = false; break; }
+      const int valid = min(kKeys, kBlock * (n_pg - 4 * j));
+      // S_t(j) complete also means tile t's earlier products (P V of stage
+      // j-1 included) have completed: none of tile t's MMAs is in flight.
+      if (!tc::mbar_wait_warp(&s_full[t], j & 1, a.status)) { ok = false; break; }
       tc::tc_fence_after();
-      const uint32_t sbuf = tmem + lane_off + t * 128 + b * 64;
-      uint32_t sr[64];
-      {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        tc::tmem_ld_32x32b_x32(sbuf, lo);
-        tc::tmem_ld_32x32b_x32(sbuf + 32, hi);
-      }
-      tc::tmem_ld_wait();
-      if (valid < kKeys) {  // warp-uniform: only the last stage of a chunk can be half full
+      uint32_t sr[128];
 #pragma unroll
-        for (int k = 32; k < 64; ++k) sr[k] = __float_as_uint(-INFINITY);
+      for (int cc = 0; cc < 4; ++cc)
+        tc::tmem_ld_32x32b_x32(sbuf + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+      tc::tmem_ld_wait();
+      if (valid < kKeys) {  // warp-uniform: only the last stage of a chunk can be partial
+#pragma unroll
+        for (int k = 32; k < 128; ++k)
+          if (k >= valid) sr[k] = __float_as_uint(-INFINITY);
       }
       float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int k = 0; k < 64; ++k) mk[k & 3] = fmaxf(mk[k & 3], __uint_as_float(sr[k]));
+      for (int k = 0; k < 128; ++k) mk[k & 3] = fmaxf(mk[k & 3], __uint_as_float(sr[k]));
       const float mt = fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])) * scale;
       const float m_new = fmaxf(m, mt);
       const bool rescale = (m == -INFINITY) || (m_new - m > kRescaleThreshold);
@@ -258,30 +248,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = m_new;
       }
       const float neg_m = -m;
-      uint32_t pk[32];
       float rk[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const float e0 = fast_exp2(fmaf(__uint_as_float(sr[2 * k]), scale, neg_m));
-        const float e1 = fast_exp2(fmaf(__uint_as_float(sr[2 * k + 1]), scale, neg_m));
+      for (int k = 0; k < 64; ++k) {  // packs in place: sr[k] <- (p_2k, p_2k+1)
+        // a quarter of the exponentials on the FMA pipe, the rest on MUFU
+        const float x0 = fmaf(__uint_as_float(sr[2 * k]), scale, neg_m);
+        const float x1 = fmaf(__uint_as_float(sr[2 * k + 1]), scale, neg_m);
+        const float e0 = (k & 3) == 3 ? poly_exp2(x0) : fast_exp2(x0);
+        const float e1 = (k & 3) == 3 ? poly_exp2(x1) : fast_exp2(x1);
         rk[k & 3] += e0 + e1;
-        pk[k] = tc::pack_bf16x2(e0, e1);
+        sr[k] = tc::pack_bf16x2(e0, e1);
       }
       l = l * alpha + ((rk[0] + rk[1]) + (rk[2] + rk[3]));
-      // No tensor-memory store while the previous P V product (a TS MMA that
-      // reads P from tensor memory) may still run: on B200 a store into
-      // another column range during that product corrupted results in
-      // testing.  The wait also makes O stable for the rescale below.
-      if (j > 0) {
-        if (!tc::mbar_wait_warp(&pv_done[t], (j - 1) & 1, a.status)) { ok = false; break; }
-        tc::tc_fence_after();
-      }
       // TMEM accesses are warp-collective, so the warp rescales together when
       // any of its rows needs it, the other rows with a factor of 1.
       const bool need = rescale && j > 0;
       if (__any_sync(0xffffffffu, need)) {
         const float f = need ? alpha : 1.f;
-        const uint32_t o_addr = tmem + lane_off + 256 + t * 128;
+        const uint32_t o_addr = tmem + lane_off + kColO + t * 128;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t ov[32];
@@ -292,8 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tmem_st_32x32b_x32(o_addr + cc * 32, ov);
         }
       }
-      // P over the first 32 columns of this S buffer (two bf16 per column).
-      tc::tmem_st_32x32b_x32(sbuf, pk);
+      // P_t(j) over the first 64 columns of S_t
+      tc::tmem_st_32x32b_x32(sbuf, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tc::tmem_st_32x32b_x32(sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tc::tmem_st_wait();
       tc::tc_fence_before();
       __syncwarp();
@@ -308,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h = g * a.G + r / kBlock;
         const int pos = r % kBlock;
         const bool single = (total <= a.ppc) || (a.max_chunks == 1);
-        const uint32_t o_addr = tmem + lane_off + 256 + t * 128;
+        const uint32_t o_addr = tmem + lane_off + kColO + t * 128;
         const float inv = 1.f / l;
         bf16* dst = a.out + ((static_cast<size_t>(s) * kBlock + pos) * a.Hq + h) * kD;
         const size_t prow_idx = ((static_cast<size_t>(s) * a.Hq + h) * a.max_chunks + c) * kBlock + pos;
