@@ -45,7 +45,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.STEP_CONFIGS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(W.STEP_CONFIGS) + [W.MASK_ATTN.name])
     ap.add_argument("--tau", type=float, default=None)
     ap.add_argument("--sub-block", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
@@ -423,8 +424,79 @@ def measure_e2e(step, cfg, tau, S, flush, dev, dist, K):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
 
 
+def run_mask_attn(args, cfg, dist: Dist):
+    """bd_block_mask_attn on the training-forward workload (2L x 2L mask)."""
+    import torch
+
+    import oracle as O
+    from decoding_bd_block_b200 import bd
+    from decoding_bd_block_b200.step import to_device
+
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    t = W.make_mask_attn_inputs(cfg)
+    q, k, v = (to_device(t[x], cfg.dtype, dev) for x in ("q", "k", "v"))
+    out = torch.empty_like(q)
+    shape = bd.make_shape(cfg.n_heads_q, cfg.n_heads_kv, cfg.head_dim, cfg.dtype)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call = lambda: bd.bd_block_mask_attn(shape, q, k, v, out, cfg.n_seqs, cfg.L, cfg.block)
+    for _ in range(args.warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    launches0 = bd.bd_kernel_launches()
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        call()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    launches = bd.bd_kernel_launches() - launches0
+    ms = dist.max(float(np.mean([e[0].elapsed_time(e[1]) for e in ev])), dev)
+    pairs = int(O.mixed_mask(cfg.L, cfg.block).sum())
+    flop = 4.0 * cfg.head_dim * cfg.n_heads_q * pairs * cfg.n_seqs
+    rows = dist.sum(float(cfg.n_seqs * 2 * cfg.L * cfg.n_heads_q), dev)
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    ach = flop / (ms / 1e3) / 1e12
+    line = {
+        "metric": "query rows attended/s (2L x 2L complementary-mask attention)",
+        "value": rows / (ms / 1e3), "unit": "query rows/s", "n_gpus": dist.world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "config": {"workload": cfg.name, "views": cfg.n_seqs, "L": cfg.L, "block": cfg.block,
+                   "n_heads_q": cfg.n_heads_q, "n_heads_kv": cfg.n_heads_kv,
+                   "head_dim": cfg.head_dim, "allowed_pairs_per_view_head": pairs,
+                   "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)"},
+        "roofline": {"kernel": "bd_block_mask_attn", "bound": "tensor", "achieved": ach,
+                     "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                     "traffic": recorded_traffic("mask_attn"),
+                     "algorithmic_flop_per_launch": flop, "peak_source": peak_kind},
+        "gpu_launches": int(launches),
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.workload == W.MASK_ATTN.name:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the reference arm times the decoding-step workloads only"}))
+            return 0
+        dist = Dist("nccl")
+        try:
+            run_mask_attn(args, W.MASK_ATTN, dist)
+        finally:
+            dist.close()
+        return 0
     cfg = W.STEP_CONFIGS[args.workload]
     tau = args.tau if args.tau is not None else cfg.taus[0]
     S = args.sub_block if args.sub_block is not None else cfg.sub_block

@@ -398,6 +398,8 @@ static cudaError_t launch_mask_t(const bd_attn_shape& sh, const void* q, const v
 cudaError_t launch_block_mask_attn(const bd_attn_shape& sh, const void* q, const void* k,
                                    const void* v, void* out, int n_seqs, int L, int block,
                                    cudaStream_t st) {
+  if (mask_attn_tc_supported(sh, L))
+    return launch_mask_attn_tc(sh, q, k, v, out, n_seqs, L, block, nullptr, st);
   const bool b = sh.dtype == BD_BF16;
   if (sh.head_dim == 64)
     return b ? launch_mask_t<bf16, 64>(sh, q, k, v, out, n_seqs, L, block, st)

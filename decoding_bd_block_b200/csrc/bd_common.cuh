@@ -163,6 +163,12 @@ cudaError_t launch_confidence_select(int dtype, int batch, int hidden, int vocab
                                      float* pmax_out, int32_t* argmax_out, void* ws,
                                      cudaStream_t st);
 
+// Tensor-core mask attention (mask_attn_tc.cu): bf16, head_dim 128, L % 128 == 0.
+bool mask_attn_tc_supported(const bd_attn_shape& sh, int L);
+cudaError_t launch_mask_attn_tc(const bd_attn_shape& sh, const void* q, const void* k,
+                                const void* v, void* out, int n_seqs, int L, int block,
+                                int32_t* status, cudaStream_t st);
+
 cudaError_t launch_block_mask_attn(const bd_attn_shape& sh, const void* q, const void* k,
                                    const void* v, void* out, int n_seqs, int L, int block,
                                    cudaStream_t st);

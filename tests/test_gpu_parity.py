@@ -247,10 +247,16 @@ def _run_mask(cfg, t):
     return out.float().cpu().numpy()
 
 
-@pytest.mark.parametrize("L,D,dtype,d", [(64, 32, "f32", 64), (96, 16, "f32", 128),
-                                         (256, 32, "bf16", 128), (128, 64, "bf16", 64)])
-def test_mask_attn_parity_small(L, D, dtype, d):
-    cfg, t = _mask_case(L, D, dtype, d=d)
+@pytest.mark.parametrize("L,D,dtype,d,Hq,Hkv", [
+    (64, 32, "f32", 64, 4, 2), (96, 16, "f32", 128, 4, 2), (128, 64, "bf16", 64, 4, 2),
+    # tensor-core path (bf16, d = 128, L % 128 == 0)
+    (256, 32, "bf16", 128, 4, 2),    # G = 2: one head pair per KV group
+    (256, 16, "bf16", 128, 6, 2),    # G = 3: a single-head last pair; many partial tiles
+    (384, 64, "bf16", 128, 12, 2),   # G = 6
+    (512, 128, "bf16", 128, 4, 1),   # D = 128: fully visible noisy diagonal tiles
+])
+def test_mask_attn_parity_small(L, D, dtype, d, Hq, Hkv):
+    cfg, t = _mask_case(L, D, dtype, d=d, Hq=Hq, Hkv=Hkv)
     got = _run_mask(cfg, t)
     ref = O.mask_attn(O.widen(t["q"], dtype), O.widen(t["k"], dtype), O.widen(t["v"], dtype), L, D)
     assert float(np.abs(got - ref).max()) <= ATOL[dtype]
