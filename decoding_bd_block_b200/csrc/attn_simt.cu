@@ -25,6 +25,8 @@ __global__ void __launch_bounds__(128) attn_prep_kernel(
     int Hkv, int d, double theta) {
   __shared__ float cs[64];
   __shared__ float sn[64];
+  griddep_wait();  // first kernel of the call: the caller's inputs are complete after this
+  griddep_launch_dependents();
   const int t = blockIdx.x, s = blockIdx.y, half = d / 2;
   const long long pos = static_cast<long long>(n_blocks[s]) * kBlock + t;
   for (int j = threadIdx.x; j < half; j += blockDim.x)
@@ -175,6 +177,8 @@ __global__ void __launch_bounds__(D) attn_merge_kernel(const int32_t* __restrict
                                                        T* __restrict__ out, int Hq, int ppc,
                                                        int max_chunks) {
   const int t = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+  griddep_wait();  // the split kernel's partials
+  griddep_launch_dependents();
   const int total = max(n_blocks[s], 0) + 1;
   if (total <= ppc) return;  // written directly by the split kernel
   const int nch = min((total + ppc - 1) / ppc, max_chunks);
@@ -267,19 +271,21 @@ static cudaError_t launch_attn_t(const bd_attn_shape& sh, const bd_kv_cache& c, 
   T* ws_blk = reinterpret_cast<T*>(w + p.off_blk);
   float* part_o = reinterpret_cast<float*>(w + p.off_o);
   float* part_ml = reinterpret_cast<float*>(w + p.off_ml);
-  attn_prep_kernel<T><<<dim3(kBlock, c.batch), 128, 0, st>>>(
-      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), c.n_blocks,
-      ws_q, ws_blk, sh.n_heads_q, sh.n_heads_kv, D, sh.rope_theta);
+  cudaError_t e = launch_pdl(attn_prep_kernel<T>, dim3(kBlock, c.batch), dim3(128), 0, st,
+                             static_cast<const T*>(q), static_cast<const T*>(k),
+                             static_cast<const T*>(v), c.n_blocks, ws_q, ws_blk, sh.n_heads_q,
+                             sh.n_heads_kv, D, sh.rope_theta);
+  if (e != cudaSuccess) return e;
   count_launches(1);
   if (p.tc) {
-    const cudaError_t e = launch_attn_tc(sh, c, p.pages_per_chunk, p.max_chunks, ws_q, ws_blk,
-                                         part_o, part_ml, out,
-                                         reinterpret_cast<int32_t*>(w + p.off_status), st);
+    e = launch_attn_tc(sh, c, p.pages_per_chunk, p.max_chunks, ws_q, ws_blk, part_o, part_ml, out,
+                       reinterpret_cast<int32_t*>(w + p.off_status), st);
     if (e != cudaSuccess) return e;
     if (p.max_chunks > 1) {
-      attn_merge_kernel<T, D><<<dim3(kBlock, sh.n_heads_q, c.batch), D, 0, st>>>(
-          c.n_blocks, part_o, part_ml, static_cast<T*>(out), sh.n_heads_q, p.pages_per_chunk,
-          p.max_chunks);
+      e = launch_pdl(attn_merge_kernel<T, D>, dim3(kBlock, sh.n_heads_q, c.batch), dim3(D), 0, st,
+                     c.n_blocks, part_o, part_ml, static_cast<T*>(out), sh.n_heads_q,
+                     p.pages_per_chunk, p.max_chunks);
+      if (e != cudaSuccess) return e;
       count_launches(1);
     }
     return cudaGetLastError();

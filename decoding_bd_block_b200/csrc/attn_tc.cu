@@ -82,7 +82,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nb = min(max(a.n_blocks[s], 0), a.max_blocks);
   const int total = nb + 1;  // cached pages + the current block
   const int p0 = c * a.ppc;
-  if (p0 >= total) return;
+  if (p0 >= total) {
+    griddep_wait();  // completes only after the prep kernel
+    return;
+  }
   const int p1 = min(total, p0 + a.ppc);
   const int n_pg = p1 - p0;
   const int n_tiles = (n_pg + 3) / 4;
@@ -117,6 +120,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::tc_fence_after();
   const uint32_t tmem = tmem_slot;
   const uint32_t sbase = tc::smem_u32(smem);
+  griddep_launch_dependents();
+  if (warp != 0) griddep_wait();  // outputs are written after the prep kernel completes
 
   if (warp == 0) {
     // ------------------------------------------------------------- producer
@@ -129,18 +134,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const uint64_t pol_kv = tc::policy_evict_first();
     const uint64_t pol_q = tc::policy_evict_last();
-    if (lane == 0) {
-      const int qrow0 = (s * a.Hq + g * a.G) * kBlock;
-      tc::mbar_arrive_expect_tx(&q_full, nq * kQTileBytes);
-      for (int t = 0; t < nq; ++t)
-        for (int dh = 0; dh < 2; ++dh)
-          tc::tma_load_2d(smem + kOffQ + t * kQTileBytes + dh * (kQTileBytes / 2), &tm_q, &q_full,
-                          dh * 64, qrow0 + 128 * t, pol_q);
-    }
+    // Cached pages were committed before this call, so the first stages of
+    // cache pages load while the prep kernel still runs; Q and the current
+    // block's page (both written by prep) load after the grid dependency.
+    bool dep = false;
+    auto wait_prep_load_q = [&]() {
+      griddep_wait();
+      dep = true;
+      if (lane == 0) {
+        const int qrow0 = (s * a.Hq + g * a.G) * kBlock;
+        tc::mbar_arrive_expect_tx(&q_full, nq * kQTileBytes);
+        for (int t = 0; t < nq; ++t)
+          for (int dh = 0; dh < 2; ++dh)
+            tc::tma_load_2d(smem + kOffQ + t * kQTileBytes + dh * (kQTileBytes / 2), &tm_q,
+                            &q_full, dh * 64, qrow0 + 128 * t, pol_q);
+      }
+      __syncwarp();
+    };
+    const bool has_blk = p1 == total;  // the chunk ends with the current block's page
     const int pg = (lane >> 2) & 3, kv = (lane >> 1) & 1, dh = lane & 1;
     int st = 0;
     uint32_t ph = 0;
     for (int j = 0; j < n_tiles; ++j) {
+      if (!dep && (j >= kStages || (has_blk && j == n_tiles - 1))) wait_prep_load_q();
       if (!tc::mbar_wait_warp(&kv_empty[st], ph ^ 1, a.status)) break;
       if (lane == 0) tc::mbar_arrive_expect_tx(&kv_full[st], 2 * kKVBytes);
       __syncwarp();
@@ -162,6 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (++st == kStages) { st = 0; ph ^= 1; }
     }
+    // Fewer tiles than stages, none holding the current block (the loop
+    // cannot stop early before `dep`: the first kStages stages are free).
+    if (!dep) wait_prep_load_q();
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -401,7 +420,9 @@ cudaError_t launch_attn_tc(const bd_attn_shape& sh, const bd_kv_cache& c, int pp
   a.out = static_cast<bf16*>(out);
   a.status = status;
   cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  attn_tc_kernel<<<dim3(max_chunks, Hkv, B), kThreads, kSmemBytes, st>>>(tm_q, tm_kv, tm_blk, a);
+  const cudaError_t e = launch_pdl(attn_tc_kernel, dim3(max_chunks, Hkv, B), dim3(kThreads),
+                                   kSmemBytes, st, tm_q, tm_kv, tm_blk, a);
+  if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
 }

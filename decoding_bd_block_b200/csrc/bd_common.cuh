@@ -53,6 +53,17 @@ __device__ __forceinline__ float poly_exp2(float x) {
   return __int_as_float(__float_as_int(p) + j * (1 << 23));
 }
 
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with launch_pdl() may start while the previous kernel of
+// the stream is still running: it must call griddep_wait() before it reads
+// anything that kernel writes (and before it writes anything that kernel
+// reads).  griddep_launch_dependents() lets the next PDL kernel start early.
+// Both are no-ops for a kernel launched the ordinary way.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // --------------------------------------------------------------- warp ops
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -107,6 +118,26 @@ int report_cuda_error(cudaError_t e);
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Launch `kern` so that it may begin before the stream's previous kernel has
+// finished (programmatic stream serialisation); see griddep_wait().  Only
+// the second and later kernels of one C-ABI call are launched this way, so
+// work enqueued before the call has always completed when they start.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 }  // namespace bd
 
 // ---------------------------------------------------------------------------
@@ -144,10 +175,11 @@ cudaError_t launch_block_attn(const bd_attn_shape& sh, const bd_kv_cache& c, con
                               cudaStream_t st);
 
 // Tensor-core LM head (select_tc.cu): persistent grid size and launcher.
+// The packed-row count is the popcount of masked[0 .. batch).
 int lmhead_tc_grid();
-cudaError_t launch_lmhead_tc(const void* rows, const void* w, const int32_t* count, int H, int V,
-                             int rows_alloc, int part_stride, float* pm, float* ps, int32_t* pa,
-                             int32_t* status, cudaStream_t st);
+cudaError_t launch_lmhead_tc(const void* rows, const void* w, const uint32_t* masked, int batch,
+                             int H, int V, int rows_alloc, int part_stride, float* pm, float* ps,
+                             int32_t* pa, int32_t* status, cudaStream_t st);
 
 struct SelectPlan {
   bool tc;           // LM head on tcgen05 (bf16)

@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(1024) gather_rows_kernel(
     int B, int H, T* __restrict__ rows, int32_t* __restrict__ posrow,
     int32_t* __restrict__ count, int rows_alloc) {
   __shared__ int red[32];
+  griddep_wait();  // first kernel of the call: the caller's inputs are complete after this
+  griddep_launch_dependents();
   const int s = blockIdx.x;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   int acc = 0;
@@ -149,6 +151,8 @@ __global__ void __launch_bounds__(1024) merge_select_kernel(
     int32_t* __restrict__ argmax_out) {
   __shared__ float sp[kBlock];
   __shared__ int stok[kBlock];
+  griddep_wait();  // the LM head's partials
+  griddep_launch_dependents();
   const int s = blockIdx.x;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t bits = masked[s];
@@ -264,22 +268,25 @@ static cudaError_t launch_select_t(int batch, int hidden, int vocab, const Selec
   float* pm = reinterpret_cast<float*>(base + p.off_pm);
   float* ps = reinterpret_cast<float*>(base + p.off_ps);
   int32_t* pa = reinterpret_cast<int32_t*>(base + p.off_pa);
-  gather_rows_kernel<T><<<batch, 1024, 0, st>>>(static_cast<const T*>(h),
-                                                static_cast<const T*>(h_prev), masked, batch,
-                                                hidden, rows, posrow, count, p.rows_alloc);
+  cudaError_t e = launch_pdl(gather_rows_kernel<T>, dim3(batch), dim3(1024), 0, st,
+                             static_cast<const T*>(h), static_cast<const T*>(h_prev), masked,
+                             batch, hidden, rows, posrow, count, p.rows_alloc);
+  if (e != cudaSuccess) return e;
   count_launches(1);
   if (p.tc) {
-    const cudaError_t e = launch_lmhead_tc(rows, w, count, hidden, vocab, p.rows_alloc, p.n_split,
-                                           pm, ps, pa, count + 1, st);
+    e = launch_lmhead_tc(rows, w, masked, batch, hidden, vocab, p.rows_alloc, p.n_split, pm, ps,
+                         pa, count + 1, st);
     if (e != cudaSuccess) return e;
   } else {
     lmhead_simt_kernel<T><<<dim3(p.n_split, p.rows_alloc / 32), 256, 0, st>>>(
         rows, static_cast<const T*>(w), count, hidden, vocab, p.n_split, pm, ps, pa);
     count_launches(1);
   }
-  merge_select_kernel<<<batch, 1024, 0, st>>>(posrow, count, masked, p.n_split, p.tc ? 1 : 0,
-                                              pm, ps, pa, tau, S, tokens, unmask, pmax_out,
-                                              argmax_out);
+  e = launch_pdl(merge_select_kernel, dim3(batch), dim3(1024), 0, st, posrow,
+                 static_cast<const int32_t*>(count), masked, p.n_split, p.tc ? 1 : 0,
+                 static_cast<const float*>(pm), static_cast<const float*>(ps),
+                 static_cast<const int32_t*>(pa), tau, S, tokens, unmask, pmax_out, argmax_out);
+  if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
 }

@@ -36,7 +36,8 @@ constexpr int kWBytes = kVTile * kKStage * 2;  // 16 KB
 constexpr int kSmemBytes = 192 * 1024;  // + ~29 KB static stays under 227 KB
 
 struct SelectTcArgs {
-  const int32_t* count;  // M (written by the gather kernel)
+  const uint32_t* masked;  // [batch] masked-position bits: M = total popcount
+  int batch;
   int H, V;
   int rows_alloc;
   int part_stride;  // partials are [row][part]
@@ -50,6 +51,7 @@ __device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
 
 __global__ void __launch_bounds__(kThreads, 1)
     lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
+                     const __grid_constant__ CUtensorMap tm_w16,
                      const __grid_constant__ CUtensorMap tm_rows, SelectTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms.
@@ -64,20 +66,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ float xpose[4][32 * 33];  // per epilogue warp: a 32 x 32 chunk, transposed
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int M = *a.count;
-  if (M <= 0) return;
+  // M, the number of packed rows, from the caller's mask bits (the gather
+  // kernel, which packs the rows, counts the same bits), so the CTA's share
+  // of the work is known before the gather kernel completes.
+  {
+    int acc = 0;
+    for (int x = threadIdx.x; x < a.batch; x += blockDim.x) acc += __popc(a.masked[x]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) red_a[0][warp] = acc;
+    __syncthreads();
+  }
+  int M = 0;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) M += red_a[0][w];
+  __syncthreads();
   const int G = (M + kMaxN - 1) / kMaxN;
-  const int R = gridDim.x / G;
+  const int R = M > 0 ? gridDim.x / G : 1;
   const int group = blockIdx.x / R, range = blockIdx.x % R;
-  if (group >= G) return;
-  const int Ng = round16((M + G - 1) / G);
+  const int Ng = M > 0 ? round16((M + G - 1) / G) : 0;
   const int row0 = group * Ng;
   const int rows_here = min(Ng, M - row0);
-  if (rows_here <= 0) return;
+  if (M <= 0 || group >= G || rows_here <= 0) {
+    griddep_wait();  // completes only after the gather kernel
+    return;
+  }
   const int N = round16(rows_here);
-  const int n_vt = (a.V + kVTile - 1) / kVTile;
-  const int t0 = static_cast<int>(static_cast<long long>(range) * n_vt / R);
-  const int t1 = static_cast<int>(static_cast<long long>(range + 1) * n_vt / R);
+  // Balanced vocab ranges in units of 16 rows: [v0, v1), split into 128-row
+  // tiles, the last one possibly short (loaded in 16-row boxes).
+  const int n_u = (a.V + 15) / 16;
+  const int v0 = 16 * static_cast<int>(static_cast<long long>(range) * n_u / R);
+  const int v1 = min(a.V, 16 * static_cast<int>(static_cast<long long>(range + 1) * n_u / R));
+  const int n_t = (v1 - v0 + kVTile - 1) / kVTile;
+  auto tile_start = [&](int it) { return v0 + it * kVTile; };
+  auto tile_rows = [&](int it) { return min(kVTile, v1 - tile_start(it)); };
   const int n_k = (a.H + kKStage - 1) / kKStage;
   const int b_bytes = N * kKStage * 2;
   const int stage_bytes = (kWBytes + b_bytes + 1023) & ~1023;
@@ -101,30 +123,63 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  griddep_launch_dependents();
+  if (warp != 0) griddep_wait();  // status and partials are written after the gather kernel
 
   if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
       tc::prefetch_tmap(&tm_w);
+      tc::prefetch_tmap(&tm_w16);
       tc::prefetch_tmap(&tm_rows);
       const uint64_t pol_w = tc::policy_evict_first();
       const uint64_t pol_r = tc::policy_evict_last();
-      int s = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      for (int t = t0; t < t1 && ok; ++t) {
-        for (int kb = 0; kb < n_k; ++kb) {
-          if (!tc::mbar_wait(&empty_bar[s], ph ^ 1, a.status)) { ok = false; break; }
-          uint8_t* st = smem + static_cast<size_t>(s) * stage_bytes;
-          tc::mbar_arrive_expect_tx(&full_bar[s], kWBytes + b_bytes);
-          tc::tma_load_2d(st, &tm_w, &full_bar[s], kb * kKStage, t * kVTile, pol_w);
-          for (int j = 0; j < N / 16; ++j)
-            tc::tma_load_2d(st + kWBytes + j * 2048, &tm_rows, &full_bar[s], kb * kKStage,
-                            row0 + 16 * j, pol_r);
-          if (++s == n_stages) { s = 0; ph ^= 1; }
+      // Stage i of the flat (vocab tile, K-slice) sequence: its W slice (a
+      // short last tile in 16-row boxes; rows past it are never used) and
+      // its packed-row slice.
+      auto w_bytes = [&](int i) {
+        const int nw = tile_rows(i / n_k);
+        return nw == kVTile ? kWBytes : (nw + 15) / 16 * 2048;
+      };
+      auto load_w = [&](int i, uint8_t* st, uint64_t* bar) {
+        const int vt = tile_start(i / n_k), kb = i % n_k;
+        if (w_bytes(i) == kWBytes) {
+          tc::tma_load_2d(st, &tm_w, bar, kb * kKStage, vt, pol_w);
+        } else {
+          for (int j = 0; j < w_bytes(i) / 2048; ++j)
+            tc::tma_load_2d(st + j * 2048, &tm_w16, bar, kb * kKStage, vt + 16 * j, pol_w);
         }
+      };
+      auto load_rows = [&](int i, uint8_t* st, uint64_t* bar) {
+        for (int j = 0; j < N / 16; ++j)
+          tc::tma_load_2d(st + kWBytes + j * 2048, &tm_rows, bar, (i % n_k) * kKStage,
+                          row0 + 16 * j, pol_r);
+      };
+      // W does not depend on the gather kernel: fill the (free) ring with W
+      // slices first, then add the packed rows once the gather completes.
+      const int n_total = n_t * n_k;
+      const int n_pre = min(n_stages, n_total);
+      for (int i = 0; i < n_pre; ++i) {
+        uint8_t* st = smem + static_cast<size_t>(i) * stage_bytes;
+        tc::mbar_arrive_expect_tx(&full_bar[i], w_bytes(i) + b_bytes);
+        load_w(i, st, &full_bar[i]);
+      }
+      griddep_wait();
+      for (int i = 0; i < n_pre; ++i)
+        load_rows(i, smem + static_cast<size_t>(i) * stage_bytes, &full_bar[i]);
+      int s = n_pre % n_stages;
+      uint32_t ph = n_pre / n_stages;
+      for (int i = n_pre; i < n_total; ++i) {
+        if (!tc::mbar_wait(&empty_bar[s], ph ^ 1, a.status)) break;
+        uint8_t* st = smem + static_cast<size_t>(s) * stage_bytes;
+        tc::mbar_arrive_expect_tx(&full_bar[s], w_bytes(i) + b_bytes);
+        load_w(i, st, &full_bar[s]);
+        load_rows(i, st, &full_bar[s]);
+        if (++s == n_stages) { s = 0; ph ^= 1; }
       }
     }
+    __syncwarp();
+    if (lane != 0) griddep_wait();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -132,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int t = t0, it = 0; t < t1 && ok; ++t, ++it) {
+      for (int it = 0; it < n_t && ok; ++it) {
         const int b = it & 1;
         const uint32_t tph = (it >> 1) & 1;
         if (!tc::mbar_wait(&tempty_bar[b], tph ^ 1, a.status)) break;
@@ -166,16 +221,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int n_chunks = N / 32 + ((N % 32) ? 1 : 0);
     bool ok = true;
-    for (int t = t0, it = 0; t < t1 && ok; ++t, ++it) {
+    for (int it = 0; it < n_t && ok; ++it) {
       const int b = it & 1;
       const uint32_t tph = (it >> 1) & 1;
       if (!tc::mbar_wait_warp(&tfull_bar[b], tph, a.status)) { ok = false; break; }
       tc::tc_fence_after();
-      const int vbase = t * kVTile + q * 32;  // vocab row of this warp's lane 0
+      const int vbase = tile_start(it) + q * 32;  // vocab row of this warp's lane 0
+      const int vend = tile_start(it) + tile_rows(it);
       // Each 32-lane x 32-column chunk goes through shared memory transposed,
       // so that thread `lane` folds column (c * 32 + lane) -- one packed row
       // -- over this warp's 32 vocab rows with plain per-thread arithmetic.
-      const bool full_tile = vbase + 32 <= a.V;
+      const bool full_tile = vbase + 32 <= vend;
       float* tb = xpose[q];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -192,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int ak[4] = {0, 0, 0, 0};
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float x = (full_tile || vbase + i < a.V) ? col[i] : -INFINITY;
+            const float x = (full_tile || vbase + i < vend) ? col[i] : -INFINITY;
             if (x > mk[i & 3]) {
               mk[i & 3] = x;
               ak[i & 3] = i;
@@ -207,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float sk[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float x = (full_tile || vbase + i < a.V) ? col[i] : -INFINITY;
+              const float x = (full_tile || vbase + i < vend) ? col[i] : -INFINITY;
               sk[i & 3] += fast_exp2(fmaf(x, kLog2e, -mls));
             }
             const float e = (sk[0] + sk[1]) + (sk[2] + sk[3]);
@@ -302,18 +358,21 @@ int lmhead_tc_grid() {
   return sms;
 }
 
-cudaError_t launch_lmhead_tc(const void* rows, const void* w, const int32_t* count, int H, int V,
-                             int rows_alloc, int part_stride, float* pm, float* ps, int32_t* pa,
-                             int32_t* status, cudaStream_t st) {
-  CUtensorMap tm_w, tm_rows;
+cudaError_t launch_lmhead_tc(const void* rows, const void* w, const uint32_t* masked, int batch,
+                             int H, int V, int rows_alloc, int part_stride, float* pm, float* ps,
+                             int32_t* pa, int32_t* status, cudaStream_t st) {
+  CUtensorMap tm_w, tm_w16, tm_rows;
   if (!make_tmap_2d(&tm_w, w, static_cast<uint64_t>(V), static_cast<uint64_t>(H), kVTile) ||
+      !make_tmap_2d(&tm_w16, w, static_cast<uint64_t>(V), static_cast<uint64_t>(H), 16) ||
       !make_tmap_2d(&tm_rows, rows, static_cast<uint64_t>(rows_alloc), static_cast<uint64_t>(H),
                     16))
     return cudaErrorInvalidValue;
-  SelectTcArgs a{count, H, V, rows_alloc, part_stride, pm, ps, pa, status};
+  SelectTcArgs a{masked, batch, H, V, rows_alloc, part_stride, pm, ps, pa, status};
   cudaFuncSetAttribute(lmhead_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        kSmemBytes + 1024);
-  lmhead_tc_kernel<<<lmhead_tc_grid(), kThreads, kSmemBytes + 1024, st>>>(tm_w, tm_rows, a);
+  const cudaError_t e = launch_pdl(lmhead_tc_kernel, dim3(lmhead_tc_grid()), dim3(kThreads),
+                                   kSmemBytes + 1024, st, tm_w, tm_w16, tm_rows, a);
+  if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
 }

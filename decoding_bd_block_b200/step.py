@@ -96,3 +96,31 @@ class DecodeStep:
             self.run_attn(stream)
         if self.sel:
             self.run_select(tau, sub_block, stream)
+
+    def capture(self, tau: float, sub_block: int, parts=("attn", "select")):
+        """Record the step's launches (the same C-ABI calls) into CUDA graphs.
+
+        Returns {part: torch.cuda.CUDAGraph}; replaying a graph re-runs that
+        call's kernels on the current buffers without host-side launch cost.
+        The cache must not grow while the graphs are in use (its block counts
+        size the attention launch).
+        """
+        graphs = {}
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.run(tau, sub_block)          # warm the launch path outside capture
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        for part in parts:
+            if (part == "attn" and not self.attn) or (part == "select" and not self.sel):
+                continue
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                if part == "attn":
+                    self.run_attn(side)
+                else:
+                    self.run_select(tau, sub_block, side)
+            graphs[part] = g
+        torch.cuda.synchronize()
+        return graphs
