@@ -110,6 +110,57 @@ __device__ __forceinline__ Stat stat_combine(Stat x, Stat y) {
   return r;
 }
 
+// ------------------------------------------ confidence-aware unmask rule
+// One sequence on one warp: lane i holds position i's mask bit (bit i of
+// `bits`), its p_max and its argmax token.  Candidates are the masked
+// positions of the lowest sub-block of S positions that still has one; every
+// candidate with p_max > tau is unmasked, or the most confident candidate
+// (lowest position on ties) when none is ("Fast-dLLM v2: Efficient
+// Block-Diffusion LLM", key design 4; Fast-dLLM v1 article, confidence-aware
+// parallel decoding).  Writes the chosen tokens, the unmask bits and, when
+// given, p_max / argmax (NaN / -1 at unmasked positions).
+__device__ __forceinline__ void select_sequence(int s, uint32_t bits, float p, int tok, float tau,
+                                                int S, int32_t* tokens, uint32_t* unmask,
+                                                float* pmax_out, int32_t* argmax_out) {
+  const int i = threadIdx.x % 32;
+  const bool is_m = (bits >> i) & 1u;
+  p = is_m ? p : 0.f;
+  tok = is_m ? tok : -1;
+  const int first = bits ? __ffs(static_cast<int>(bits)) - 1 : 0;
+  const int k0 = (first / S) * S;
+  const bool cand = is_m && i >= k0 && i < k0 + S;
+  const uint32_t above = __ballot_sync(0xffffffffu, cand && p > tau);
+  uint32_t U = above;
+  if (!above) {
+    float bp = cand ? p : -1.f;
+    int bi = cand ? i : 32;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float op = __shfl_xor_sync(0xffffffffu, bp, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (op > bp || (op == bp && oi < bi)) {
+        bp = op;
+        bi = oi;
+      }
+    }
+    U = (bi < 32) ? (1u << bi) : 0u;
+  }
+  if ((U >> i) & 1u) tokens[s * kBlock + i] = tok;
+  if (i == 0) unmask[s] = U;
+  if (pmax_out) pmax_out[s * kBlock + i] = is_m ? p : __int_as_float(0x7fc00000);
+  if (argmax_out) argmax_out[s * kBlock + i] = is_m ? tok : -1;
+}
+
+// "No decision" for sequence s (a bounded wait gave up): nothing is
+// unmasked, p_max is NaN and the token -2.  Lane i of one warp writes position i.
+__device__ __forceinline__ void no_decision_sequence(int s, uint32_t* unmask, float* pmax_out,
+                                                     int32_t* argmax_out) {
+  const int i = threadIdx.x % 32;
+  if (i == 0) unmask[s] = 0u;
+  if (pmax_out) pmax_out[s * kBlock + i] = __int_as_float(0x7fc00000);
+  if (argmax_out) argmax_out[s * kBlock + i] = -2;
+}
+
 // Process-wide count of kernels enqueued by the library (bd_kernel_launches).
 void count_launches(int n);
 // Records a CUDA error for bd_last_cuda_error_string(); returns BD_ERR_CUDA
@@ -182,12 +233,24 @@ cudaError_t launch_lmhead_tc(const void* rows, const void* w, const uint32_t* ma
                              int32_t* pa, int32_t* status, cudaStream_t st);
 
 struct SelectPlan {
+  bool fused;        // one kernel, rows resident in shared memory (select_fused.cu)
   bool tc;           // LM head on tcgen05 (bf16)
   int n_split;       // vocab splits (partials per row)
   int rows_alloc;    // packed-row capacity (>= 32 * batch, padded)
   size_t off_rows, off_posrow, off_count, off_pm, off_ps, off_pa, total;
 };
 SelectPlan plan_confidence_select(int dtype, int batch, int hidden, int vocab);
+
+// Single-kernel select (select_fused.cu): bf16, one sequence.  Partials are
+// [32 positions][select_fused_part_stride()]; header points at the zeroed
+// workspace header ([1] status, [2] arrivals, [3] tile counter), left zero.
+bool select_fused_supported(int dtype, int batch, int hidden);
+int select_fused_part_stride();
+cudaError_t launch_select_fused(int hidden, int vocab, const void* h, const void* h_prev,
+                                const void* w, const uint32_t* masked, float tau, int sub_block,
+                                int32_t* tokens, uint32_t* unmask, float* pmax_out,
+                                int32_t* argmax_out, float* pm, float* ps, int32_t* pa,
+                                int32_t* header, cudaStream_t st);
 cudaError_t launch_confidence_select(int dtype, int batch, int hidden, int vocab,
                                      const SelectPlan& p, const void* h, const void* h_prev,
                                      const void* w, const uint32_t* masked, float tau,

@@ -1,0 +1,392 @@
+// bd_confidence_select in ONE kernel for a single sequence: token shift, LM
+// head with online softmax statistics, and the confidence-aware unmask
+// ("Fast-dLLM v2: Efficient Block-Diffusion LLM", key designs 2-4; Fast-dLLM
+// v1 article, confidence-aware parallel decoding).
+//
+// Persistent grid, one CTA per SM:
+//
+//   * The token shift needs no gather: the MMA's N operand is the block's 32
+//     hidden rows h[0..31] followed by h_prev, fetched by TMA straight from
+//     the caller's buffers (N = 48: 32 + a 16-row slot of which one row is
+//     used).  Column j < 31 scores position j + 1 and column 32 position 0;
+//     column 31 (the next block's first position) and 33.. are ignored.
+//   * Vocab tiles of 128 rows: each CTA takes tile blockIdx.x, then further
+//     tiles from an atomic counter, so SMs that get more HBM bandwidth take
+//     more tiles and all finish within about one tile of each other.  (A
+//     tile costs n_k ring stages whatever its rows, and the stream runs
+//     latency-bound on bytes in flight, so smaller tiles at the end would
+//     run at a fraction of the bandwidth.)  Warp 0 streams the tile's W
+//     slices (128 x 64, 16 KB) with the matching 48 x 64 operand slice
+//     through a TMA ring; warp 1 issues tcgen05.mma into one of two
+//     64-column TMEM accumulators; warps 2-5 fold the other into running
+//     (max, sum exp, argmax) per column.
+//   * Each CTA writes one partial per masked position; the last CTA to
+//     finish (an arrival counter) merges them, applies the unmask rule and
+//     zeroes the counters and the status word for the next call.
+#include "lmhead_common.cuh"
+
+namespace bd {
+namespace {
+
+using lmh::kKStage;
+using lmh::kVTile;
+using lmh::kWBytes;
+
+constexpr int kThreads = 192;                         // 6 warps
+constexpr int kN = 48;                                // MMA N
+constexpr int kBBytes = kN * kKStage * 2;             // 6 KB operand slice
+constexpr int kStageBytes = kWBytes + kBBytes;        // 22 KB, a multiple of 1 KB
+constexpr int kSmemBytes = 192 * 1024;
+constexpr int kStages = kSmemBytes / kStageBytes;     // 8
+constexpr uint32_t kTmemCols = 128;                   // two 64-column accumulators
+constexpr int kSlots = 8;                             // published tile indices in flight
+constexpr int kHpRow = 32;                            // operand row of h_prev
+
+static_assert(kStageBytes % 1024 == 0, "stages must keep the 1 KB swizzle alignment");
+
+struct FusedArgs {
+  const uint32_t* masked;  // [1]
+  int H, V;
+  float tau;
+  int S;
+  int32_t* tokens;
+  uint32_t* unmask;
+  float* pmax_out;
+  int32_t* argmax_out;
+  float* pm;  // partials [32 positions][part_stride]
+  float* ps;
+  int32_t* pa;
+  int part_stride;    // >= gridDim.x, a multiple of 4
+  int32_t* status;    // 0 between calls; a bounded wait that gave up sets it
+  uint32_t* arrivals; // 0 between calls
+  int32_t* tile_ctr;  // 0 between calls
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    select_fused_kernel(const __grid_constant__ CUtensorMap tm_w,
+                        const __grid_constant__ CUtensorMap tm_w16,
+                        const __grid_constant__ CUtensorMap tm_h,
+                        const __grid_constant__ CUtensorMap tm_hp, FusedArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  __shared__ uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ uint64_t tfull_bar[2], tempty_bar[2];
+  __shared__ uint64_t tile_bar[kSlots], tile_free[kSlots];
+  __shared__ int tile_q[kSlots];
+  __shared__ uint32_t tmem_slot;
+  __shared__ float red_m[4][64], red_s[4][64];
+  __shared__ int red_a[4][64];
+  __shared__ float xpose[4][32 * 33];
+  __shared__ float sp[kBlock];
+  __shared__ int stok[kBlock];
+  __shared__ int pos_of[kBlock];  // position of the r-th masked bit
+  __shared__ int s_last;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_k = (a.H + kKStage - 1) / kKStage;
+  const int R = gridDim.x;
+  const int n_tiles = (a.V + kVTile - 1) / kVTile;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&full_bar[s], 1);
+      tc::mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&tfull_bar[b], 1);
+      tc::mbar_init(&tempty_bar[b], 4);
+    }
+    for (int i = 0; i < kSlots; ++i) {
+      tc::mbar_init(&tile_bar[i], 1);
+      tc::mbar_init(&tile_free[i], 5);  // the MMA issuer and the 4 epilogue warps
+    }
+    tc::fence_barrier_init();
+  }
+  // Operand rows 33..47 are never loaded: zero them once in every stage.
+  for (int x = threadIdx.x; x < kStages * (kN - kHpRow - 1) * 8; x += kThreads) {
+    const int s = x / ((kN - kHpRow - 1) * 8), rem = x % ((kN - kHpRow - 1) * 8);
+    const int row = kHpRow + 1 + rem / 8, c = rem % 8;
+    tc::st_shared_v4(tc::smem_u32(smem + s * kStageBytes + kWBytes + row * 128 + c * 16), 0u, 0u,
+                     0u, 0u);
+  }
+  tc::fence_proxy_async();
+  if (warp == 1) tc::tmem_alloc(&tmem_slot, kTmemCols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  griddep_wait();  // first kernel of the call: the caller's inputs are complete after this
+  griddep_launch_dependents();
+  const uint32_t bits = a.masked[0];
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_w);
+      tc::prefetch_tmap(&tm_w16);
+      tc::prefetch_tmap(&tm_h);
+      tc::prefetch_tmap(&tm_hp);
+      const uint64_t pol_w = tc::policy_evict_first();
+      const uint64_t pol_h = tc::policy_evict_last();
+      int next = bits ? blockIdx.x : n_tiles;  // the first tile needs no counter
+      int s = 0;
+      uint32_t ph = 0;
+      for (int it = 0;; ++it) {
+        const int t = next < n_tiles ? next : -1;
+        const int slot = it % kSlots;
+        if (!tc::mbar_wait(&tile_free[slot], ((it / kSlots) & 1) ^ 1, a.status)) break;
+        tile_q[slot] = t;
+        tc::mbar_arrive(&tile_bar[slot]);  // release: consumers read tile_q after their wait
+        if (t < 0) break;
+        next = R + atomicAdd(a.tile_ctr, 1);  // the next tile, fetched while this one streams
+        const int vt = t * kVTile, nw = min(kVTile, a.V - vt);
+        const int nbox = nw == kVTile ? 0 : (nw + 15) / 16;
+        const int w_bytes = nbox ? nbox * 2048 : kWBytes;
+        bool ok = true;
+        for (int kb = 0; kb < n_k; ++kb) {
+          if (!tc::mbar_wait(&empty_bar[s], ph ^ 1, a.status)) { ok = false; break; }
+          uint8_t* st = smem + static_cast<size_t>(s) * kStageBytes;
+          uint64_t* bar = &full_bar[s];
+          // 16 + 16 rows of h and the one row of h_prev
+          tc::mbar_arrive_expect_tx(bar, w_bytes + (2 * 16 + 1) * 128);
+          if (!nbox) tc::tma_load_2d(st, &tm_w, bar, kb * kKStage, vt, pol_w);
+          for (int j = 0; j < nbox; ++j)  // short last tile: accumulator rows past it are ignored
+            tc::tma_load_2d(st + j * 2048, &tm_w16, bar, kb * kKStage, vt + 16 * j, pol_w);
+          tc::tma_load_2d(st + kWBytes, &tm_h, bar, kb * kKStage, 0, pol_h);
+          tc::tma_load_2d(st + kWBytes + 16 * 128, &tm_h, bar, kb * kKStage, 16, pol_h);
+          tc::tma_load_2d(st + kWBytes + kHpRow * 128, &tm_hp, bar, kb * kKStage, 0, pol_h);
+          if (++s == kStages) { s = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16_f32(kVTile, kN);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        const int slot = it % kSlots;
+        if (!tc::mbar_wait(&tile_bar[slot], (it / kSlots) & 1, a.status)) break;
+        const int t = tile_q[slot];
+        tc::mbar_arrive(&tile_free[slot]);
+        if (t < 0) break;
+        const int b = it & 1;
+        if (!tc::mbar_wait(&tempty_bar[b], ((it >> 1) & 1) ^ 1, a.status)) break;
+        tc::tc_fence_after();
+        const uint32_t d = tmem + b * 64;
+        for (int kb = 0; kb < n_k; ++kb) {
+          if (!tc::mbar_wait(&full_bar[s], ph, a.status)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t sa = tc::smem_u32(smem + static_cast<size_t>(s) * kStageBytes);
+          const uint32_t sb = sa + kWBytes;
+#pragma unroll
+          for (int kk = 0; kk < kKStage / 16; ++kk)
+            tc::mma_bf16_ss(d, tc::sdesc_kmajor_sw128(sa + kk * 32),
+                            tc::sdesc_kmajor_sw128(sb + kk * 32), idesc, (kb | kk) != 0);
+          tc::mma_commit(&empty_bar[s]);
+          if (++s == kStages) { s = 0; ph ^= 1; }
+        }
+        tc::mma_commit(&tfull_bar[b]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    lmh::Run run0 = lmh::run_empty(), run1 = lmh::run_empty();
+    for (int it = 0;; ++it) {
+      const int slot = it % kSlots;
+      if (!tc::mbar_wait_warp(&tile_bar[slot], (it / kSlots) & 1, a.status)) break;
+      const int t = tile_q[slot];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tile_free[slot]);
+      if (t < 0) break;
+      const int b = it & 1;
+      if (!tc::mbar_wait_warp(&tfull_bar[b], (it >> 1) & 1, a.status)) break;
+      tc::tc_fence_after();
+      const int vbase = t * kVTile + q * 32, vend = min(a.V, t * kVTile + kVTile);
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * 64;
+      lmh::fold_chunk(taddr, xpose[q], lane, vbase, vend, run0);       // h[0..31]
+      lmh::fold_chunk(taddr + 32, xpose[q], lane, vbase, vend, run1);  // h_prev, unused
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty_bar[b]);
+    }
+    red_m[q][lane] = run0.m;
+    red_s[q][lane] = run0.s;
+    red_a[q][lane] = run0.a;
+    red_m[q][32 + lane] = run1.m;
+    red_s[q][32 + lane] = run1.s;
+    red_a[q][32 + lane] = run1.a;
+    tc::named_bar_sync(1, 128);
+    const int col = threadIdx.x - 64;
+    const int pos = col == kHpRow ? 0 : col + 1;  // position this column scores
+    if ((col < kBlock - 1 || col == kHpRow) && ((bits >> pos) & 1u)) {
+      Stat st = stat_empty();
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq)
+        st = stat_combine(st, Stat{red_m[qq][col], red_s[qq][col], red_a[qq][col]});
+      const size_t idx = static_cast<size_t>(pos) * a.part_stride + blockIdx.x;
+      a.pm[idx] = st.m;
+      a.ps[idx] = st.s;
+      a.pa[idx] = st.a;
+      __threadfence();
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
+
+  // ------------------------------------------- last CTA: merge and select
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(a.arrivals, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // Partials of the masked positions into shared memory (the ring is idle
+  // now), all loads in flight at once, then one warp per position reduces.
+  const int P = gridDim.x, PS = a.part_stride;
+  const int M = __popc(bits);
+  if (warp == 0 && ((bits >> lane) & 1u)) pos_of[__popc(bits & ((1u << lane) - 1u))] = lane;
+  __syncthreads();
+  float* lm = reinterpret_cast<float*>(smem);
+  float* ls = lm + kBlock * PS;
+  int* la = reinterpret_cast<int*>(ls + kBlock * PS);
+  {
+    const int vec_per_row = PS / 4;
+    const int total = M * vec_per_row;
+    for (int x0 = threadIdx.x; x0 < total; x0 += kThreads * 8) {
+      uint4 vm[8], vs[8], va[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int x = x0 + u * kThreads;
+        if (x < total) {
+          const int r = x / vec_per_row, c = x % vec_per_row;
+          const size_t g = static_cast<size_t>(pos_of[r]) * PS + 4 * c;
+          vm[u] = __ldcg(reinterpret_cast<const uint4*>(a.pm + g));
+          vs[u] = __ldcg(reinterpret_cast<const uint4*>(a.ps + g));
+          va[u] = __ldcg(reinterpret_cast<const uint4*>(a.pa + g));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int x = x0 + u * kThreads;
+        if (x < total) {
+          const int r = x / vec_per_row, c = x % vec_per_row;
+          reinterpret_cast<uint4*>(lm + r * PS)[c] = vm[u];
+          reinterpret_cast<uint4*>(ls + r * PS)[c] = vs[u];
+          reinterpret_cast<uint4*>(la + r * PS)[c] = va[u];
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // Eight lanes per position: the max and the lowest index attaining it
+  // first, then the sum of exp(m_k - max) s_k, one exponential per part.
+  for (int r0 = warp * 4; r0 < M; r0 += kThreads / 8) {
+    const int r = r0 + lane / 8, j = lane % 8;
+    const bool live = r < M;
+    const float* rm = lm + (live ? r : 0) * PS;
+    const float* rs = ls + (live ? r : 0) * PS;
+    const int* ra = la + (live ? r : 0) * PS;
+    float mx = -INFINITY;
+    int am = 0x7fffffff;
+    for (int k = j; live && k < P; k += 8) {
+      const float m = rm[k];
+      if (m > mx || (m == mx && ra[k] < am)) {
+        mx = m;
+        am = ra[k];
+      }
+    }
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) {
+      const float om = __shfl_xor_sync(0xffffffffu, mx, o);
+      const int oa = __shfl_xor_sync(0xffffffffu, am, o);
+      if (om > mx || (om == mx && oa < am)) {
+        mx = om;
+        am = oa;
+      }
+    }
+    float sum = 0.f;
+    for (int k = j; live && k < P; k += 8)
+      if (rm[k] != -INFINITY) sum += rs[k] * expf(rm[k] - mx);
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (live && j == 0) {
+      sp[r] = sum > 0.f ? 1.f / sum : 0.f;  // p_max = exp(max - max) / sum
+      stok[r] = am;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const bool is_m = (bits >> lane) & 1u;
+    const int r = __popc(bits & ((1u << lane) - 1u));
+    if (__ldcg(a.status) != 0)
+      no_decision_sequence(0, a.unmask, a.pmax_out, a.argmax_out);
+    else
+      select_sequence(0, bits, is_m ? sp[r] : 0.f, is_m ? stok[r] : -1, a.tau, a.S, a.tokens,
+                      a.unmask, a.pmax_out, a.argmax_out);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {  // ready for the next call on this workspace
+    *a.arrivals = 0u;
+    *a.tile_ctr = 0;
+    *a.status = 0;
+  }
+}
+
+}  // namespace
+
+bool select_fused_supported(int dtype, int batch, int hidden) {
+  return dtype == BD_BF16 && batch == 1 && hidden % 8 == 0 &&
+         kBlock * select_fused_part_stride() * 12 <= kSmemBytes;
+}
+
+int select_fused_part_stride() { return (lmh::sm_count() + 3) / 4 * 4; }
+
+cudaError_t launch_select_fused(int hidden, int vocab, const void* h, const void* h_prev,
+                                const void* w, const uint32_t* masked, float tau, int sub_block,
+                                int32_t* tokens, uint32_t* unmask, float* pmax_out,
+                                int32_t* argmax_out, float* pm, float* ps, int32_t* pa,
+                                int32_t* header, cudaStream_t st) {
+  CUtensorMap tm_w, tm_w16, tm_h, tm_hp;
+  if (!lmh::make_tmap_2d(&tm_w, w, static_cast<uint64_t>(vocab), static_cast<uint64_t>(hidden),
+                         kVTile) ||
+      !lmh::make_tmap_2d(&tm_w16, w, static_cast<uint64_t>(vocab), static_cast<uint64_t>(hidden),
+                         16) ||
+      !lmh::make_tmap_2d(&tm_h, h, kBlock, static_cast<uint64_t>(hidden), 16) ||
+      !lmh::make_tmap_2d(&tm_hp, h_prev, 1, static_cast<uint64_t>(hidden), 1))
+    return cudaErrorInvalidValue;
+  FusedArgs a{};
+  a.masked = masked;
+  a.H = hidden;
+  a.V = vocab;
+  a.tau = tau;
+  a.S = sub_block;
+  a.tokens = tokens;
+  a.unmask = unmask;
+  a.pmax_out = pmax_out;
+  a.argmax_out = argmax_out;
+  a.pm = pm;
+  a.ps = ps;
+  a.pa = pa;
+  a.part_stride = select_fused_part_stride();
+  a.status = header + 1;
+  a.arrivals = reinterpret_cast<uint32_t*>(header + 2);
+  a.tile_ctr = header + 3;
+  cudaFuncSetAttribute(select_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       kSmemBytes + 1024);
+  const cudaError_t e = launch_pdl(select_fused_kernel, dim3(lmh::sm_count()), dim3(kThreads),
+                                   kSmemBytes + 1024, st, tm_w, tm_w16, tm_h, tm_hp, a);
+  if (e != cudaSuccess) return e;
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace bd

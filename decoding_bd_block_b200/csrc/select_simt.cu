@@ -157,11 +157,7 @@ __global__ void __launch_bounds__(1024) merge_select_kernel(
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t bits = masked[s];
   if (count[1] != 0) {
-    if (threadIdx.x < kBlock) {
-      if (threadIdx.x == 0) unmask[s] = 0u;
-      if (pmax_out) pmax_out[s * kBlock + threadIdx.x] = __int_as_float(0x7fc00000);
-      if (argmax_out) argmax_out[s * kBlock + threadIdx.x] = -2;
-    }
+    if (warp == 0) no_decision_sequence(s, unmask, pmax_out, argmax_out);
     return;
   }
   const int parts = grouped ? n_split / ((count[0] + 255) / 256) : n_split;
@@ -185,34 +181,7 @@ __global__ void __launch_bounds__(1024) merge_select_kernel(
   }
   __syncthreads();
   if (warp != 0) return;
-  const int i = lane;
-  const bool is_m = (bits >> i) & 1u;
-  const float p = is_m ? sp[i] : 0.f;
-  const int tok = is_m ? stok[i] : -1;
-  // Candidates: masked positions of the lowest sub-block that has one.
-  const int first = bits ? __ffs(static_cast<int>(bits)) - 1 : 0;
-  const int k0 = (first / S) * S;
-  const bool cand = is_m && i >= k0 && i < k0 + S;
-  const uint32_t above = __ballot_sync(0xffffffffu, cand && p > tau);
-  uint32_t U = above;
-  if (!above) {
-    float bp = cand ? p : -1.f;
-    int bi = cand ? i : 32;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float op = __shfl_xor_sync(0xffffffffu, bp, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (op > bp || (op == bp && oi < bi)) {
-        bp = op;
-        bi = oi;
-      }
-    }
-    U = (bi < 32) ? (1u << bi) : 0u;
-  }
-  if ((U >> i) & 1u) tokens[s * kBlock + i] = tok;
-  if (i == 0) unmask[s] = U;
-  if (pmax_out) pmax_out[s * kBlock + i] = is_m ? p : __int_as_float(0x7fc00000);
-  if (argmax_out) argmax_out[s * kBlock + i] = is_m ? tok : -1;
+  select_sequence(s, bits, sp[lane], stok[lane], tau, S, tokens, unmask, pmax_out, argmax_out);
 }
 
 // -------------------------------------------------------------- host side
@@ -225,8 +194,12 @@ static bool use_tc(int dtype, int batch) {
 SelectPlan plan_confidence_select(int dtype, int batch, int hidden, int vocab) {
   SelectPlan p{};
   p.rows_alloc = static_cast<int>(align_up(static_cast<size_t>(batch) * kBlock, 256));
+  p.fused = select_fused_supported(dtype, batch, hidden);
   p.tc = use_tc(dtype, batch);
-  if (p.tc) {
+  if (p.fused) {
+    p.rows_alloc = kBlock;  // partials per position of the one sequence
+    p.n_split = select_fused_part_stride();
+  } else if (p.tc) {
     p.n_split = lmhead_tc_grid();
   } else {
     const int vtiles = (vocab + 63) / 64;
@@ -238,12 +211,15 @@ SelectPlan plan_confidence_select(int dtype, int batch, int hidden, int vocab) {
   }
   const size_t es = dtype == BD_BF16 ? 2 : 4;
   size_t off = 0;
+  // Header, zero between calls: [0] = M, [1] = status word of the
+  // tensor-core kernels, [2] = CTA arrivals and [3] = vocab-tile counter of
+  // the single-kernel path.
+  p.off_count = off;
+  off = align_up(off + 16, 256);
   p.off_rows = off;
-  off = align_up(off + static_cast<size_t>(p.rows_alloc) * hidden * es, 256);
+  if (!p.fused) off = align_up(off + static_cast<size_t>(p.rows_alloc) * hidden * es, 256);
   p.off_posrow = off;
-  off = align_up(off + static_cast<size_t>(batch) * kBlock * 4, 256);
-  p.off_count = off;  // [0] = M, [1] = status word of the tensor-core kernel
-  off = align_up(off + 8, 256);
+  if (!p.fused) off = align_up(off + static_cast<size_t>(batch) * kBlock * 4, 256);
   const size_t part = static_cast<size_t>(p.n_split) * p.rows_alloc * 4;
   p.off_pm = off;
   off = align_up(off + part, 256);
@@ -268,6 +244,9 @@ static cudaError_t launch_select_t(int batch, int hidden, int vocab, const Selec
   float* pm = reinterpret_cast<float*>(base + p.off_pm);
   float* ps = reinterpret_cast<float*>(base + p.off_ps);
   int32_t* pa = reinterpret_cast<int32_t*>(base + p.off_pa);
+  if (p.fused)
+    return launch_select_fused(hidden, vocab, h, h_prev, w, masked, tau, S, tokens, unmask,
+                               pmax_out, argmax_out, pm, ps, pa, count, st);
   cudaError_t e = launch_pdl(gather_rows_kernel<T>, dim3(batch), dim3(1024), 0, st,
                              static_cast<const T*>(h), static_cast<const T*>(h_prev), masked,
                              batch, hidden, rows, posrow, count, p.rows_alloc);

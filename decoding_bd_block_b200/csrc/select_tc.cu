@@ -20,19 +20,20 @@
 //     running (max, sum, argmax) that lane (column mod 32) keeps.
 //   * At the end the 4 epilogue warps combine through shared memory and the
 //     CTA writes one (max, sum, argmax) partial per row of its group.
-#include "bd_common.cuh"
-#include "tc_common.cuh"
+#include "lmhead_common.cuh"
 
 namespace bd {
 namespace {
 
-constexpr int kThreads = 192;      // 6 warps
-constexpr int kVTile = 128;        // vocab rows per MMA (M)
-constexpr int kKStage = 64;        // hidden elements per stage (128 B rows)
-constexpr int kMaxN = 256;         // packed rows per group (MMA N)
+using lmh::kKStage;
+using lmh::kVTile;
+using lmh::kWBytes;
+using lmh::round16;
+
+constexpr int kThreads = 192;  // 6 warps
+constexpr int kMaxN = 256;     // packed rows per group (MMA N)
 constexpr int kMaxStages = 12;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kWBytes = kVTile * kKStage * 2;  // 16 KB
 constexpr int kSmemBytes = 192 * 1024;  // + ~29 KB static stays under 227 KB
 
 struct SelectTcArgs {
@@ -46,8 +47,6 @@ struct SelectTcArgs {
   int32_t* pa;
   int32_t* status;
 };
-
-__device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
 
 __global__ void __launch_bounds__(kThreads, 1)
     lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_w,
@@ -93,13 +92,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int N = round16(rows_here);
   // Balanced vocab ranges in units of 16 rows: [v0, v1), split into 128-row
-  // tiles, the last one possibly short (loaded in 16-row boxes).
+  // tiles.  The first tile takes the remainder (rem rows, loaded in 16-row
+  // boxes when short), so that its small loads overlap the full tiles
+  // streaming behind it instead of trailing at the end of the range.
   const int n_u = (a.V + 15) / 16;
   const int v0 = 16 * static_cast<int>(static_cast<long long>(range) * n_u / R);
   const int v1 = min(a.V, 16 * static_cast<int>(static_cast<long long>(range + 1) * n_u / R));
   const int n_t = (v1 - v0 + kVTile - 1) / kVTile;
-  auto tile_start = [&](int it) { return v0 + it * kVTile; };
-  auto tile_rows = [&](int it) { return min(kVTile, v1 - tile_start(it)); };
+  const int rem = v1 - v0 - (n_t - 1) * kVTile;  // rows of tile 0 (1..128 when n_t > 0)
+  auto tile_start = [&](int it) { return it == 0 ? v0 : v0 + rem + (it - 1) * kVTile; };
+  auto tile_rows = [&](int it) { return it == 0 ? rem : kVTile; };
   const int n_k = (a.H + kKStage - 1) / kKStage;
   const int b_bytes = N * kKStage * 2;
   const int stage_bytes = (kWBytes + b_bytes + 1023) & ~1023;
@@ -211,14 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    float run_m[8], run_s[8];
-    int run_a[8];
+    lmh::Run run[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      run_m[c] = -INFINITY;
-      run_s[c] = 0.f;
-      run_a[c] = 0x7fffffff;
-    }
+    for (int c = 0; c < 8; ++c) run[c] = lmh::run_empty();
     const int n_chunks = N / 32 + ((N % 32) ? 1 : 0);
     bool ok = true;
     for (int it = 0; it < n_t && ok; ++it) {
@@ -228,58 +225,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_after();
       const int vbase = tile_start(it) + q * 32;  // vocab row of this warp's lane 0
       const int vend = tile_start(it) + tile_rows(it);
-      // Each 32-lane x 32-column chunk goes through shared memory transposed,
-      // so that thread `lane` folds column (c * 32 + lane) -- one packed row
-      // -- over this warp's 32 vocab rows with plain per-thread arithmetic.
-      const bool full_tile = vbase + 32 <= vend;
-      float* tb = xpose[q];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        if (c < n_chunks) {
-          uint32_t r[32];
-          tc::tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + b * kMaxN + c * 32,
-                                 r);
-          tc::tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) tb[j * 33 + lane] = __uint_as_float(r[j]);
-          __syncwarp();
-          const float* col = tb + lane * 33;
-          float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          int ak[4] = {0, 0, 0, 0};
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float x = (full_tile || vbase + i < vend) ? col[i] : -INFINITY;
-            if (x > mk[i & 3]) {
-              mk[i & 3] = x;
-              ak[i & 3] = i;
-            }
-          }
-          float mx = fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3]));
-          int am = 32;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) am = (mk[k] == mx && ak[k] < am) ? ak[k] : am;
-          if (mx != -INFINITY) {
-            const float mls = mx * kLog2e;
-            float sk[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float x = (full_tile || vbase + i < vend) ? col[i] : -INFINITY;
-              sk[i & 3] += fast_exp2(fmaf(x, kLog2e, -mls));
-            }
-            const float e = (sk[0] + sk[1]) + (sk[2] + sk[3]);
-            const int arg = vbase + am;
-            if (mx > run_m[c]) {
-              run_s[c] = run_s[c] * fast_exp2((run_m[c] - mx) * kLog2e) + e;
-              run_m[c] = mx;
-              run_a[c] = arg;
-            } else {
-              run_s[c] += e * fast_exp2((mx - run_m[c]) * kLog2e);
-              if (mx == run_m[c] && arg < run_a[c]) run_a[c] = arg;
-            }
-          }
-          __syncwarp();
-        }
-      }
+      for (int c = 0; c < 8; ++c)
+        if (c < n_chunks)
+          lmh::fold_chunk(tmem + (static_cast<uint32_t>(q * 32) << 16) + b * kMaxN + c * 32,
+                          xpose[q], lane, vbase, vend, run[c]);
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&tempty_bar[b]);
@@ -289,9 +239,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; c < 8; ++c) {
       const int col = c * 32 + lane;
       if (col < N) {
-        red_m[q][col] = run_m[c];
-        red_s[q][col] = run_s[c];
-        red_a[q][col] = run_a[c];
+        red_m[q][col] = run[c].m;
+        red_s[q][col] = run[c].s;
+        red_a[q][col] = run[c].a;
       }
     }
     tc::named_bar_sync(1, 128);
@@ -312,59 +262,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// 2-D bf16 tensor [rows][cols] (row-major), tile box [box_rows][64 cols],
-// 128-byte swizzle, zero fill outside the tensor.
-bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                  uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {64, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
-int lmhead_tc_grid() {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
-  return sms;
-}
+int lmhead_tc_grid() { return lmh::sm_count(); }
 
 cudaError_t launch_lmhead_tc(const void* rows, const void* w, const uint32_t* masked, int batch,
                              int H, int V, int rows_alloc, int part_stride, float* pm, float* ps,
                              int32_t* pa, int32_t* status, cudaStream_t st) {
   CUtensorMap tm_w, tm_w16, tm_rows;
-  if (!make_tmap_2d(&tm_w, w, static_cast<uint64_t>(V), static_cast<uint64_t>(H), kVTile) ||
-      !make_tmap_2d(&tm_w16, w, static_cast<uint64_t>(V), static_cast<uint64_t>(H), 16) ||
-      !make_tmap_2d(&tm_rows, rows, static_cast<uint64_t>(rows_alloc), static_cast<uint64_t>(H),
+  if (!lmh::make_tmap_2d(&tm_w, w, static_cast<uint64_t>(V), static_cast<uint64_t>(H), kVTile) ||
+      !lmh::make_tmap_2d(&tm_w16, w, static_cast<uint64_t>(V), static_cast<uint64_t>(H), 16) ||
+      !lmh::make_tmap_2d(&tm_rows, rows, static_cast<uint64_t>(rows_alloc), static_cast<uint64_t>(H),
                     16))
     return cudaErrorInvalidValue;
   SelectTcArgs a{masked, batch, H, V, rows_alloc, part_stride, pm, ps, pa, status};

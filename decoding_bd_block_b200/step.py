@@ -77,7 +77,7 @@ class DecodeStep:
             self.pmax = torch.empty((B, BLOCK), dtype=torch.float32, device=device)
             self.argmax = torch.empty((B, BLOCK), dtype=torch.int32, device=device)
             n = bd.bd_confidence_select_workspace_size(dt, B, cfg.hidden, cfg.vocab)
-            self.sel_ws = torch.empty(n, dtype=torch.uint8, device=device)
+            self.sel_ws = torch.zeros(n, dtype=torch.uint8, device=device)  # header must start zero
             self.n_scored = int(sum(bin(int(b)).count("1") for b in self.masked_host))
 
     def run_attn(self, stream=None):

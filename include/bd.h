@@ -160,10 +160,14 @@ BD_API int bd_block_attn(const bd_attn_shape* shape, const bd_kv_cache* cache,
  *                position, -1 elsewhere
  * sub_block must divide 32; 0 <= tau; hidden % 8 == 0; h, h_prev and w_lm
  * 16-byte aligned.  Workspace: bd_confidence_select_workspace_size() bytes,
- * 256-byte aligned.  bf16 runs the LM head on the tensor cores (tcgen05):
- * if one of its bounded waits ever gives up (it never should), the call
- * reports "no decision" for the whole batch: unmask_bits 0, p_max NaN and
- * argmax -2. */
+ * 256-byte aligned, its first 256 bytes zero before the first call that
+ * uses it (cudaMemset once when it is allocated): the library keeps a
+ * status word and an arrival counter there, which every call leaves ready
+ * for the next, so the caller must not write to them between calls, nor
+ * use one workspace in two calls that may run at the same time.  bf16 runs
+ * the LM head on the tensor cores (tcgen05): if one of its bounded waits
+ * ever gives up (it never should), the call reports "no decision" for the
+ * whole batch: unmask_bits 0, p_max NaN and argmax -2. */
 BD_API int bd_confidence_select_workspace_size(int32_t dtype, int32_t batch,
                                         int32_t hidden, int32_t vocab,
                                         size_t* bytes);

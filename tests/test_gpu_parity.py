@@ -191,6 +191,15 @@ SELECT_CASES = [
                          seed=97), 0.0, 8),
     (dataclasses.replace(W.TINY_F32, name="f32_subblock1", batch=4, n_masked=0,
                          masked_range=(0, 32), seed=98), 0.9, 1),
+    # batch 1: the single-kernel path with the rows resident in shared memory
+    (dataclasses.replace(W.QWEN15B_STEP, name="fused_n16_h520_vocab_tail", vocab=1000, hidden=520,
+                         n_masked=9, seed=101), 0.5, 4),
+    (dataclasses.replace(W.QWEN15B_STEP, name="fused_all_masked_h2304", vocab=3000, hidden=2304,
+                         n_masked=32, seed=102), 0.9, 8),
+    (dataclasses.replace(W.QWEN15B_STEP, name="fused_none_masked", vocab=1000, hidden=256,
+                         n_masked=0, seed=103), 0.9, 8),
+    (dataclasses.replace(W.QWEN15B_STEP, name="fused_one_masked_v65536", vocab=65536, hidden=1536,
+                         n_masked=1, seed=104), 0.9, 8),
 ]
 
 
@@ -211,19 +220,29 @@ def test_confidence_select_parity(case):
             assert bin(int(step.unmask[b].item()) & 0xFFFFFFFF).count("1") == want
 
 
-def test_select_idempotent_and_masked_untouched():
-    cfg = dataclasses.replace(W.QWEN15B_STEP, batch=3, vocab=4096, seed=99)
+@pytest.mark.parametrize("batch", [1, 3])  # single-kernel and three-kernel paths
+def test_select_idempotent_and_masked_untouched(batch):
+    cfg = dataclasses.replace(W.QWEN15B_STEP, batch=batch, vocab=4096, seed=99)
     _, s, step = _step(cfg, attn=False)
     step.run_select(0.9, 8)
     t1, u1 = step.tokens.clone(), step.unmask.clone()
-    step.run_select(0.9, 8)
+    p1 = step.pmax.clone()
+    for _ in range(3):  # the workspace header (status, arrivals) is reset by every call
+        step.run_select(0.9, 8)
     torch.cuda.synchronize()
     assert torch.equal(t1, step.tokens) and torch.equal(u1, step.unmask)
+    assert torch.equal(p1.isnan(), step.pmax.isnan())
+    # vocab tiles go to whichever CTA asks first, so the order in which the
+    # exp-sums are added, and with it the last bits of p_max, may vary
+    torch.testing.assert_close(torch.nan_to_num(p1), torch.nan_to_num(step.pmax), rtol=1e-5,
+                               atol=0)
+    hdr = step.sel_ws[:16].view(torch.int32).cpu()
+    assert hdr[1] == 0 and hdr[2] == 0 and hdr[3] == 0
     assert torch.equal(step.masked.cpu(), torch.from_numpy(s["masked_bits"].view(np.int32)))
     tin = step.tokens_in.cpu().numpy()
     tout = step.tokens.cpu().numpy()
     un = step.unmask.cpu().numpy().view(np.uint32)
-    for b in range(3):
+    for b in range(batch):
         for i in range(32):
             if not (int(un[b]) >> i) & 1:
                 assert tout[b, i] == tin[b, i]
