@@ -16,42 +16,116 @@
 namespace bd {
 
 // ------------------------------------------------------------- prep kernel
-// grid (32, batch); rotated q -> ws_q [B][Hq][32][d]; rotated k_blk and v_blk
-// -> ws_blk [B][2][Hkv][32][d] (a cache page of the current block).
-template <typename T>
-__global__ void __launch_bounds__(128) attn_prep_kernel(
+// 8 consecutive elements of a row, converted to fp32 (one 16-byte load for
+// bf16, two for fp32; rows are 16-byte aligned).
+struct Vec8 {
+  float f[8];
+};
+__device__ __forceinline__ Vec8 load8(const bf16* p) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+  Vec8 r;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = __bfloat1622float2(h[i]);
+    r.f[2 * i] = x.x;
+    r.f[2 * i + 1] = x.y;
+  }
+  return r;
+}
+__device__ __forceinline__ Vec8 load8(const float* p) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  return Vec8{{a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w}};
+}
+__device__ __forceinline__ void store8(bf16* p, const Vec8& v) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v.f[2 * i], v.f[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+__device__ __forceinline__ void store8(float* p, const Vec8& v) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v.f[0], v.f[1], v.f[2], v.f[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v.f[4], v.f[5], v.f[6], v.f[7]);
+}
+
+// grid (32, batch), 256 threads; one CTA per position t of sequence s.
+// Rotated q -> ws_q [B][Hq][32][d]; rotated k_blk and v_blk -> ws_blk
+// [B][2][Hkv][32][d] (a cache page of the current block).  Work items of 8
+// elements: q and k items carry the 8 matching elements of both halves of
+// the rotation pairs (j, j + d/2); v items are plain copies.  Each thread
+// issues the loads of its first two items before the rotation table is
+// built, so the item loads and the double-precision angles overlap.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) attn_prep_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const int32_t* __restrict__ n_blocks, T* __restrict__ ws_q, T* __restrict__ ws_blk, int Hq,
-    int Hkv, int d, double theta) {
-  __shared__ float cs[64];
-  __shared__ float sn[64];
+    int Hkv, RopeFreq freq) {
+  constexpr int C = D / 16;  // items per (head, row): 8-element groups of the first half
+  __shared__ float cs[D / 2];
+  __shared__ float sn[D / 2];
   griddep_wait();  // first kernel of the call: the caller's inputs are complete after this
   griddep_launch_dependents();
-  const int t = blockIdx.x, s = blockIdx.y, half = d / 2;
+  const int t = blockIdx.x, s = blockIdx.y;
+  const int n_q = Hq * C, n_k = Hkv * C, n_v = Hkv * 2 * C;
+  const int total = n_q + n_k + n_v;
+  const size_t row = static_cast<size_t>(s) * kBlock + t;
+  // item -> (source, destination) of its (first) 8 elements
+  auto src_of = [&](int it) -> const T* {
+    if (it < n_q) return q + (row * Hq + it / C) * D + (it % C) * 8;
+    it -= n_q;
+    if (it < n_k) return k + (row * Hkv + it / C) * D + (it % C) * 8;
+    it -= n_k;
+    return v + (row * Hkv + it / (2 * C)) * D + (it % (2 * C)) * 8;
+  };
+  auto dst_of = [&](int it) -> T* {
+    if (it < n_q) return ws_q + ((static_cast<size_t>(s) * Hq + it / C) * kBlock + t) * D + (it % C) * 8;
+    it -= n_q;
+    if (it < n_k)
+      return ws_blk + ((static_cast<size_t>(s) * 2 + 0) * Hkv + it / C) * kBlock * D + t * D +
+             (it % C) * 8;
+    it -= n_k;
+    return ws_blk + ((static_cast<size_t>(s) * 2 + 1) * Hkv + it / (2 * C)) * kBlock * D + t * D +
+           (it % (2 * C)) * 8;
+  };
+  auto process = [&](int it, const Vec8& lo, const Vec8& hi) {
+    T* dst = dst_of(it);
+    if (it >= n_q + n_k) {
+      store8(dst, lo);
+      return;
+    }
+    const int j0 = (it % C) * 8;
+    Vec8 a, b;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      a.f[e] = lo.f[e] * cs[j0 + e] - hi.f[e] * sn[j0 + e];
+      b.f[e] = hi.f[e] * cs[j0 + e] + lo.f[e] * sn[j0 + e];
+    }
+    store8(dst, a);
+    store8(dst + D / 2, b);
+  };
+  Vec8 lo[2], hi[2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int it = threadIdx.x + u * blockDim.x;
+    if (it < total) {
+      const T* src = src_of(it);
+      lo[u] = load8(src);
+      if (it < n_q + n_k) hi[u] = load8(src + D / 2);
+    }
+  }
   const long long pos = static_cast<long long>(n_blocks[s]) * kBlock + t;
-  for (int j = threadIdx.x; j < half; j += blockDim.x)
-    rope_cos_sin(pos, rope_inv_freq(j, d, theta), &cs[j], &sn[j]);
+  for (int j = threadIdx.x; j < D / 2; j += blockDim.x) rope_cos_sin(pos, freq.inv[j], &cs[j], &sn[j]);
   __syncthreads();
-  for (int idx = threadIdx.x; idx < Hq * half; idx += blockDim.x) {
-    const int h = idx / half, j = idx % half;
-    const T* src = q + ((static_cast<size_t>(s) * kBlock + t) * Hq + h) * d;
-    const float x1 = to_f32(src[j]), x2 = to_f32(src[j + half]);
-    T* dst = ws_q + ((static_cast<size_t>(s) * Hq + h) * kBlock + t) * d;
-    dst[j] = from_f32<T>(x1 * cs[j] - x2 * sn[j]);
-    dst[j + half] = from_f32<T>(x2 * cs[j] + x1 * sn[j]);
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int it = threadIdx.x + u * blockDim.x;
+    if (it < total) process(it, lo[u], hi[u]);
   }
-  for (int idx = threadIdx.x; idx < Hkv * half; idx += blockDim.x) {
-    const int g = idx / half, j = idx % half;
-    const T* src = k + ((static_cast<size_t>(s) * kBlock + t) * Hkv + g) * d;
-    const float x1 = to_f32(src[j]), x2 = to_f32(src[j + half]);
-    T* dst = ws_blk + ((static_cast<size_t>(s) * 2 + 0) * Hkv + g) * kBlock * d + t * d;
-    dst[j] = from_f32<T>(x1 * cs[j] - x2 * sn[j]);
-    dst[j + half] = from_f32<T>(x2 * cs[j] + x1 * sn[j]);
-  }
-  for (int idx = threadIdx.x; idx < Hkv * d; idx += blockDim.x) {
-    const int g = idx / d, c = idx % d;
-    ws_blk[((static_cast<size_t>(s) * 2 + 1) * Hkv + g) * kBlock * d + t * d + c] =
-        v[((static_cast<size_t>(s) * kBlock + t) * Hkv + g) * d + c];
+  for (int it = threadIdx.x + 2 * blockDim.x; it < total; it += blockDim.x) {
+    const T* src = src_of(it);
+    const Vec8 l = load8(src);
+    process(it, l, it < n_q + n_k ? load8(src + D / 2) : l);
   }
 }
 
@@ -169,7 +243,9 @@ __global__ void __launch_bounds__(256) attn_split_simt_kernel(
   }
 }
 
-// grid (32, Hq, batch), D threads: merge the chunks of one output row.
+// grid (32, Hq, batch), D threads: merge the chunks of one output row.  The
+// chunks' (m, l, O) are read eight at a time, all loads in flight, and
+// folded into a running (max, sum, acc) in base-2 exponent units.
 template <typename T, int D>
 __global__ void __launch_bounds__(D) attn_merge_kernel(const int32_t* __restrict__ n_blocks,
                                                        const float* __restrict__ part_o,
@@ -183,14 +259,36 @@ __global__ void __launch_bounds__(D) attn_merge_kernel(const int32_t* __restrict
   if (total <= ppc) return;  // written directly by the split kernel
   const int nch = min((total + ppc - 1) / ppc, max_chunks);
   const size_t base = (static_cast<size_t>(s) * Hq + h) * max_chunks;
-  float M = -INFINITY;
-  for (int c = 0; c < nch; ++c) M = fmaxf(M, part_ml[((base + c) * kBlock + t) * 2]);
-  float L = 0.f, acc = 0.f;
-  for (int c = 0; c < nch; ++c) {
-    const size_t row = (base + c) * kBlock + t;
-    const float w = exp2f(part_ml[row * 2] - M);
-    L += part_ml[row * 2 + 1] * w;
-    acc += part_o[row * D + threadIdx.x] * w;
+  float M = -INFINITY, L = 0.f, acc = 0.f;
+  for (int c0 = 0; c0 < nch; c0 += 8) {
+    float m[8], l[8], o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c = c0 + u;
+      m[u] = -INFINITY;
+      l[u] = 0.f;
+      o[u] = 0.f;
+      if (c < nch) {
+        const size_t r = (base + c) * kBlock + t;
+        const float2 ml = reinterpret_cast<const float2*>(part_ml)[r];
+        m[u] = ml.x;
+        l[u] = ml.y;
+        o[u] = part_o[r * D + threadIdx.x];
+      }
+    }
+    float Mn = M;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) Mn = fmaxf(Mn, m[u]);
+    const float sc = M == -INFINITY ? 0.f : exp2f(M - Mn);
+    L *= sc;
+    acc *= sc;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float w = m[u] == -INFINITY ? 0.f : exp2f(m[u] - Mn);
+      L += l[u] * w;
+      acc += o[u] * w;
+    }
+    M = Mn;
   }
   out[((static_cast<size_t>(s) * kBlock + t) * Hq + h) * D + threadIdx.x] = from_f32<T>(acc / L);
 }
@@ -271,10 +369,12 @@ static cudaError_t launch_attn_t(const bd_attn_shape& sh, const bd_kv_cache& c, 
   T* ws_blk = reinterpret_cast<T*>(w + p.off_blk);
   float* part_o = reinterpret_cast<float*>(w + p.off_o);
   float* part_ml = reinterpret_cast<float*>(w + p.off_ml);
-  cudaError_t e = launch_pdl(attn_prep_kernel<T>, dim3(kBlock, c.batch), dim3(128), 0, st,
+  RopeFreq freq;
+  rope_freq_table(D, sh.rope_theta, &freq);
+  cudaError_t e = launch_pdl(attn_prep_kernel<T, D>, dim3(kBlock, c.batch), dim3(256), 0, st,
                              static_cast<const T*>(q), static_cast<const T*>(k),
                              static_cast<const T*>(v), c.n_blocks, ws_q, ws_blk, sh.n_heads_q,
-                             sh.n_heads_kv, D, sh.rope_theta);
+                             sh.n_heads_kv, freq);
   if (e != cudaSuccess) return e;
   count_launches(1);
   if (p.tc) {

@@ -1,6 +1,7 @@
 // C-ABI entry points of libbd: host-side validation, workspace planning and
 // dispatch to the kernels.  Nothing here allocates device memory.
 #include <atomic>
+#include <cmath>
 #include <cstring>
 #include <vector>
 
@@ -9,6 +10,11 @@
 namespace bd {
 static std::atomic<long long> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+void rope_freq_table(int d, double theta, RopeFreq* f) {
+  for (int j = 0; j < 64; ++j)
+    f->inv[j] = j < d / 2 ? std::pow(theta, -2.0 * j / static_cast<double>(d)) : 0.0;
+}
 }  // namespace bd
 
 namespace {
@@ -140,6 +146,8 @@ int bd_block_attn(const bd_attn_shape* sh, const bd_kv_cache* c, const void* q, 
   if (st) return st;
   if ((st = check_cache(sh, c))) return st;
   if (!q || !k || !v || !out) return BD_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, static_cast<const void*>(out)})
+    if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return BD_ERR_INVALID_ARG;
   const bd::AttnPlan p = bd::plan_block_attn(*sh, *c);
   if (p.total > 0 && (!ws || ws_bytes < p.total)) return BD_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return BD_ERR_WORKSPACE;

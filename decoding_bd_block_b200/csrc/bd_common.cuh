@@ -90,6 +90,13 @@ __device__ __forceinline__ double rope_inv_freq(int j, int d, double theta) {
   return pow(theta, -2.0 * static_cast<double>(j) / static_cast<double>(d));
 }
 
+// theta^(-2j/d) for j < d/2, computed on the host in double precision and
+// passed by value, so that a kernel needs no pow.
+struct RopeFreq {
+  double inv[64];
+};
+void rope_freq_table(int d, double theta, RopeFreq* f);
+
 // ------------------------------------------------- (max, sum, argmax) triple
 // Running softmax statistics of a set of logits: m = max, s = sum exp(l - m),
 // a = lowest index attaining m.  combine() is associative and commutative.

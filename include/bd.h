@@ -123,7 +123,8 @@ BD_API int bd_cache_commit(const bd_attn_shape* shape, bd_kv_cache* cache,
  *   out    device, [batch][32][n_heads_q][head_dim], written
  * q and k_blk are rotated at positions P..P+31 (P = 32 * n_blocks[s]);
  * out = softmax(q K^T / sqrt(head_dim)) V over [cached keys ; block keys].
- * batch is cache->batch.  Workspace: bd_block_attn_workspace_size() bytes,
+ * q, k_blk, v_blk and out are 16-byte aligned (BD_ERR_INVALID_ARG
+ * otherwise).  batch is cache->batch.  Workspace: bd_block_attn_workspace_size() bytes,
  * 256-byte aligned; its size depends on n_blocks_host, so ask again after
  * the cache grows. */
 BD_API int bd_block_attn_workspace_size(const bd_attn_shape* shape,
