@@ -309,12 +309,11 @@ def run_ours(args, cfg, tau, S, dist: Dist):
         step.run_select(tau, S)
     per_step = bd.bd_kernel_launches() - n0
     sel_launches = per_step - (n1 - n0)
-    graphs = None if args.eager else step.capture(tau, S)
+    graphs = None if args.eager else step.capture(tau, S, parts=("step", "attn", "select"))
     for _ in range(2):
         flush.zero_()
         if graphs:
-            for g in graphs.values():
-                g.replay()
+            graphs["step"].replay()
         else:
             step.run(tau, S)
     torch.cuda.synchronize(dev)
@@ -326,7 +325,7 @@ def run_ours(args, cfg, tau, S, dist: Dist):
         pass
     sampler = ClockSampler(uuid)
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     launches0 = bd.bd_kernel_launches()
     dist.barrier()
     torch.cuda.synchronize(dev)
@@ -334,21 +333,34 @@ def run_ours(args, cfg, tau, S, dist: Dist):
     for i in range(K):
         flush.zero_()
         ev[i][0].record(stream)
-        if step.attn:
-            graphs["attn"].replay() if graphs else step.run_attn()
+        if graphs:
+            graphs["step"].replay()
+        else:
+            step.run(tau, S)
         ev[i][1].record(stream)
-        if step.sel:
-            graphs["select"].replay() if graphs else step.run_select(tau, S)
-        ev[i][2].record(stream)
     torch.cuda.synchronize(dev)
     dist.barrier()
     t_wall1 = time.time()
+    # Per-call breakdown, outside the timed region: each call on its own
+    # (one graph per call), L2 flushed before each step as above.
+    n_bd = max(10, K // 4)
+    evb = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_bd)]
+    for i in range(n_bd):
+        flush.zero_()
+        evb[i][0].record(stream)
+        if step.attn:
+            graphs["attn"].replay() if graphs else step.run_attn()
+        evb[i][1].record(stream)
+        if step.sel:
+            graphs["select"].replay() if graphs else step.run_select(tau, S)
+        evb[i][2].record(stream)
+    torch.cuda.synchronize(dev)
     launches = per_step * K if graphs else bd.bd_kernel_launches() - launches0
     clocks = sampler.stop(t_wall0, t_wall1)
 
-    t_attn = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
-    t_sel = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    t_step = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
+    t_attn = [evb[i][0].elapsed_time(evb[i][1]) for i in range(n_bd)]
+    t_sel = [evb[i][1].elapsed_time(evb[i][2]) for i in range(n_bd)]
+    t_step = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     ms_rank = float(np.mean(t_step))
     ms = dist.max(ms_rank, dev)
     n_scored = step.n_scored if step.sel else 0

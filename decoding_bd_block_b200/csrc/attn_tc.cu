@@ -31,6 +31,8 @@
 //
 // The chunk's (m, l, O) go to the workspace for attn_merge_kernel, or --
 // when one chunk covers the whole sequence -- O / l straight to the output.
+#include <cstring>
+
 #include "bd_common.cuh"
 #include "tc_common.cuh"
 
@@ -67,7 +69,9 @@ struct AttnTcArgs {
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
-                   const __grid_constant__ CUtensorMap tm_blk, AttnTcArgs a) {
+                   const __grid_constant__ CUtensorMap tm_blk,
+                   const __grid_constant__ CUtensorMap tm_out,
+                   const __grid_constant__ CUtensorMap tm_po, AttnTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -309,36 +313,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && tc::mbar_wait_warp(&pv_done[t], (n_tiles - 1) & 1, a.status)) {
       tc::tc_fence_after();
       if (32 * (r / 32) < a.R) {
+        // The warp's 32 rows are the 32 positions of one query head h.  O
+        // goes out by TMA tile stores from the warp's 8 KB slice of its
+        // query tile's Q buffer (free once the tile's last product is done),
+        // written in the store's 128-byte-swizzled layout: bf16 O / l as two
+        // (64 d x 32 positions) boxes of `out`, or the fp32 chunk partial as
+        // four (32 d x 32 positions) boxes of the partial buffer.
         const int h = g * a.G + r / kBlock;
         const int pos = r % kBlock;
         const bool single = (total <= a.ppc) || (a.max_chunks == 1);
         const uint32_t o_addr = tmem + lane_off + kColO + t * 128;
         const float inv = 1.f / l;
-        bf16* dst = a.out + ((static_cast<size_t>(s) * kBlock + pos) * a.Hq + h) * kD;
-        const size_t prow_idx = ((static_cast<size_t>(s) * a.Hq + h) * a.max_chunks + c) * kBlock + pos;
-        float* po = a.part_o + prow_idx * kD;
+        const size_t prow0 = ((static_cast<size_t>(s) * a.Hq + h) * a.max_chunks + c) * kBlock;
+        const size_t prow_idx = prow0 + pos;
+        uint8_t* stg = smem + kOffQ + t * kQTileBytes + q * 8192;
+        if (single) {
+#pragma unroll 1
+          for (int dh = 0; dh < 2; ++dh) {  // 64 d per box
+            uint8_t* box = stg + dh * 4096;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t ov[32];
-          tc::tmem_ld_32x32b_x32(o_addr + cc * 32, ov);
-          tc::tmem_ld_wait();
-          if (single) {
-            uint32_t pkd[16];
+            for (int half = 0; half < 2; ++half) {
+              uint32_t ov[32];
+              tc::tmem_ld_32x32b_x32(o_addr + dh * 64 + half * 32, ov);
+              tc::tmem_ld_wait();
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
-              pkd[k] = tc::pack_bf16x2(__uint_as_float(ov[2 * k]) * inv,
-                                       __uint_as_float(ov[2 * k + 1]) * inv);
-            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              d4[k] = make_uint4(pkd[4 * k], pkd[4 * k + 1], pkd[4 * k + 2], pkd[4 * k + 3]);
-          } else {
-            float4* p4 = reinterpret_cast<float4*>(po + cc * 32);
+              for (int k = 0; k < 4; ++k) {  // 8 bf16 = one 16-byte chunk
+                uint4 v;
+                v.x = tc::pack_bf16x2(__uint_as_float(ov[8 * k + 0]) * inv, __uint_as_float(ov[8 * k + 1]) * inv);
+                v.y = tc::pack_bf16x2(__uint_as_float(ov[8 * k + 2]) * inv, __uint_as_float(ov[8 * k + 3]) * inv);
+                v.z = tc::pack_bf16x2(__uint_as_float(ov[8 * k + 4]) * inv, __uint_as_float(ov[8 * k + 5]) * inv);
+                v.w = tc::pack_bf16x2(__uint_as_float(ov[8 * k + 6]) * inv, __uint_as_float(ov[8 * k + 7]) * inv);
+                const int chunk = half * 4 + k;
+                *reinterpret_cast<uint4*>(box + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = v;
+              }
+            }
+          }
+          tc::fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            tc::tma_store_3d(&tm_out, stg, 0, h, s * kBlock);
+            tc::tma_store_3d(&tm_out, stg + 4096, 64, h, s * kBlock);
+            tc::bulk_commit();
+            tc::bulk_wait_read<0>();
+          }
+          __syncwarp();
+        } else {
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {  // 32 fp32 per box
+            uint8_t* box = stg + (cc & 1) * 4096;
+            if (cc >= 2) {  // the box's previous store must have read it
+              if (lane == 0) tc::bulk_wait_read<1>();
+              __syncwarp();
+            }
+            uint32_t ov[32];
+            tc::tmem_ld_32x32b_x32(o_addr + cc * 32, ov);
+            tc::tmem_ld_wait();
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              p4[k] = make_float4(__uint_as_float(ov[4 * k]), __uint_as_float(ov[4 * k + 1]),
-                                  __uint_as_float(ov[4 * k + 2]), __uint_as_float(ov[4 * k + 3]));
+              *reinterpret_cast<uint4*>(box + lane * 128 + ((k ^ (lane & 7)) << 4)) =
+                  make_uint4(ov[4 * k], ov[4 * k + 1], ov[4 * k + 2], ov[4 * k + 3]);
+            tc::fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tc::tma_store_2d(&tm_po, box, cc * 32, static_cast<int>(prow0));
+              tc::bulk_commit();
+            }
           }
+          if (lane == 0) tc::bulk_wait_read<0>();
+          __syncwarp();
         }
         if (!single) {
           a.part_ml[prow_idx * 2 + 0] = m;
@@ -383,6 +425,33 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_row
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output [rows][heads][128] bf16 viewed as (d, head, row): box = 32 rows of
+// one head, 64 d wide, 128-byte swizzle (tile stores).
+bool make_tmap_out(CUtensorMap* m, const void* base, uint64_t rows, uint32_t heads) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), heads, rows};
+  const cuuint64_t strides[2] = {kD * 2, static_cast<cuuint64_t>(heads) * kD * 2};
+  const cuuint32_t box[3] = {64, 1, kBlock};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 partial O [rows][128]: box = 32 rows x 32 floats (128 bytes), 128-byte swizzle.
+bool make_tmap_part(CUtensorMap* m, const void* base, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), rows};
+  const cuuint64_t strides[1] = {kD * 4};
+  const cuuint32_t box[2] = {32, kBlock};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool attn_tc_supported(const bd_attn_shape& sh) {
@@ -396,12 +465,17 @@ cudaError_t launch_attn_tc(const bd_attn_shape& sh, const bd_kv_cache& c, int pp
                            const void* ws_q, const void* ws_blk, float* part_o, float* part_ml,
                            void* out, int32_t* status, cudaStream_t st) {
   const int B = c.batch, Hq = sh.n_heads_q, Hkv = sh.n_heads_kv;
-  CUtensorMap tm_q, tm_kv, tm_blk;
+  CUtensorMap tm_q, tm_kv, tm_blk, tm_out, tm_po;
   const uint64_t kv_rows = static_cast<uint64_t>(c.n_pages) * 2 * Hkv * kBlock;
   if (kv_rows >= (1ull << 31)) return cudaErrorInvalidValue;
   if (!make_tmap(&tm_q, ws_q, static_cast<uint64_t>(B) * Hq * kBlock, 128) ||
       !make_tmap(&tm_kv, c.pages, kv_rows, kBlock) ||
-      !make_tmap(&tm_blk, ws_blk, static_cast<uint64_t>(B) * 2 * Hkv * kBlock, kBlock))
+      !make_tmap(&tm_blk, ws_blk, static_cast<uint64_t>(B) * 2 * Hkv * kBlock, kBlock) ||
+      !make_tmap_out(&tm_out, out, static_cast<uint64_t>(B) * kBlock, Hq))
+    return cudaErrorInvalidValue;
+  std::memset(&tm_po, 0, sizeof(tm_po));  // unused unless a sequence spans several chunks
+  if (max_chunks > 1 &&
+      !make_tmap_part(&tm_po, part_o, static_cast<uint64_t>(B) * Hq * max_chunks * kBlock))
     return cudaErrorInvalidValue;
   AttnTcArgs a{};
   a.page_table = c.page_table;
@@ -421,7 +495,7 @@ cudaError_t launch_attn_tc(const bd_attn_shape& sh, const bd_kv_cache& c, int pp
   a.status = status;
   cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   const cudaError_t e = launch_pdl(attn_tc_kernel, dim3(max_chunks, Hkv, B), dim3(kThreads),
-                                   kSmemBytes, st, tm_q, tm_kv, tm_blk, a);
+                                   kSmemBytes, st, tm_q, tm_kv, tm_blk, tm_out, tm_po, a);
   if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();

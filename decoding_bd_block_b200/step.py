@@ -102,8 +102,10 @@ class DecodeStep:
 
         Returns {part: torch.cuda.CUDAGraph}; replaying a graph re-runs that
         call's kernels on the current buffers without host-side launch cost.
-        The cache must not grow while the graphs are in use (its block counts
-        size the attention launch).
+        Part "step" holds both calls in one graph, so the select call's first
+        kernel is chained to the attention call's last one.  The cache must
+        not grow while the graphs are in use (its block counts size the
+        attention launch).
         """
         graphs = {}
         side = torch.cuda.Stream()
@@ -119,8 +121,10 @@ class DecodeStep:
             with torch.cuda.graph(g, stream=side):
                 if part == "attn":
                     self.run_attn(side)
-                else:
+                elif part == "select":
                     self.run_select(tau, sub_block, side)
+                else:
+                    self.run(tau, sub_block, side)
             graphs[part] = g
         torch.cuda.synchronize()
         return graphs
