@@ -10,16 +10,19 @@
 //     the caller's buffers (N = 48: 32 + a 16-row slot of which one row is
 //     used).  Column j < 31 scores position j + 1 and column 32 position 0;
 //     column 31 (the next block's first position) and 33.. are ignored.
-//   * Vocab tiles of 128 rows: each CTA takes tile blockIdx.x, then further
-//     tiles from an atomic counter, so SMs that get more HBM bandwidth take
-//     more tiles and all finish within about one tile of each other.  (A
-//     tile costs n_k ring stages whatever its rows, and the stream runs
-//     latency-bound on bytes in flight, so smaller tiles at the end would
-//     run at a fraction of the bandwidth.)  Warp 0 streams the tile's W
-//     slices (128 x 64, 16 KB) with the matching 48 x 64 operand slice
-//     through a TMA ring; warp 1 issues tcgen05.mma into one of two
-//     64-column TMEM accumulators; warps 2-5 fold the other into running
-//     (max, sum exp, argmax) per column.
+//   * Vocab tiles of TR <= 128 rows, TR chosen by the host so that the tile
+//     count is close to a multiple of the grid (151936 rows over 148 CTAs:
+//     115-row tiles, 9 per CTA, instead of 1187 = 8 x 148 + 3 tiles of 128
+//     that leave three CTAs a whole tile behind).  Each CTA takes tile
+//     blockIdx.x, then further tiles from an atomic counter, so SMs that get
+//     more HBM bandwidth take more tiles.  (A tile costs n_k ring stages
+//     whatever its rows and the stream runs latency-bound on bytes in
+//     flight, so tiles much smaller than 128 rows would lose bandwidth.)
+//     Warp 0 streams the tile's W slices (TR x 64) with the matching 48 x 64
+//     operand slice through a TMA ring; warp 1 issues tcgen05.mma (M = 128:
+//     accumulator rows past TR are ignored) into one of two 64-column TMEM
+//     accumulators; warps 2-5 fold the other into running (max, sum exp,
+//     argmax) per column.
 //   * Each CTA writes one partial per masked position; the last CTA to
 //     finish (an arrival counter) merges them, applies the unmask rule and
 //     zeroes the counters and the status word for the next call.
@@ -30,19 +33,23 @@ namespace {
 
 using lmh::kKStage;
 using lmh::kVTile;
-using lmh::kWBytes;
 
 constexpr int kThreads = 192;                         // 6 warps
 constexpr int kN = 48;                                // MMA N
 constexpr int kBBytes = kN * kKStage * 2;             // 6 KB operand slice
-constexpr int kStageBytes = kWBytes + kBBytes;        // 22 KB, a multiple of 1 KB
 constexpr int kSmemBytes = 192 * 1024;
-constexpr int kStages = kSmemBytes / kStageBytes;     // 8
+constexpr int kMaxStages = 12;
+constexpr int kMinTileRows = 64;
 constexpr uint32_t kTmemCols = 128;                   // two 64-column accumulators
 constexpr int kSlots = 8;                             // published tile indices in flight
 constexpr int kHpRow = 32;                            // operand row of h_prev
 
-static_assert(kStageBytes % 1024 == 0, "stages must keep the 1 KB swizzle alignment");
+// Stage = W slice (TR rows x 128 bytes, rounded up to 1 KB) + operand slice.
+// The MMA reads 128 rows (16 KB) of A from the stage's start, which the W
+// region plus the operand slice always covers (hence W region >= 10 KB).
+__host__ __device__ constexpr int stage_w_bytes(int tr) {
+  return (tr * 128 + 1023) / 1024 * 1024 < 10240 ? 10240 : (tr * 128 + 1023) / 1024 * 1024;
+}
 
 struct FusedArgs {
   const uint32_t* masked;  // [1]
@@ -57,6 +64,7 @@ struct FusedArgs {
   float* ps;
   int32_t* pa;
   int part_stride;    // >= gridDim.x, a multiple of 4
+  int tile_rows;      // TR: W rows per vocab tile (the W tensor map's box)
   int32_t* status;    // 0 between calls; a bounded wait that gave up sets it
   uint32_t* arrivals; // 0 between calls
   int32_t* tile_ctr;  // 0 between calls
@@ -64,13 +72,12 @@ struct FusedArgs {
 
 __global__ void __launch_bounds__(kThreads, 1)
     select_fused_kernel(const __grid_constant__ CUtensorMap tm_w,
-                        const __grid_constant__ CUtensorMap tm_w16,
                         const __grid_constant__ CUtensorMap tm_h,
                         const __grid_constant__ CUtensorMap tm_hp, FusedArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  __shared__ uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ uint64_t full_bar[kMaxStages], empty_bar[kMaxStages];
   __shared__ uint64_t tfull_bar[2], tempty_bar[2];
   __shared__ uint64_t tile_bar[kSlots], tile_free[kSlots];
   __shared__ int tile_q[kSlots];
@@ -86,10 +93,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_k = (a.H + kKStage - 1) / kKStage;
   const int R = gridDim.x;
-  const int n_tiles = (a.V + kVTile - 1) / kVTile;
+  const int TR = a.tile_rows;
+  const int n_tiles = (a.V + TR - 1) / TR;
+  const int w_region = stage_w_bytes(TR);
+  const int stage_bytes = w_region + kBBytes;
+  int n_stages = kSmemBytes / stage_bytes;
+  n_stages = n_stages > kMaxStages ? kMaxStages : n_stages;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < n_stages; ++s) {
       tc::mbar_init(&full_bar[s], 1);
       tc::mbar_init(&empty_bar[s], 1);
     }
@@ -104,10 +116,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_barrier_init();
   }
   // Operand rows 33..47 are never loaded: zero them once in every stage.
-  for (int x = threadIdx.x; x < kStages * (kN - kHpRow - 1) * 8; x += kThreads) {
+  for (int x = threadIdx.x; x < n_stages * (kN - kHpRow - 1) * 8; x += kThreads) {
     const int s = x / ((kN - kHpRow - 1) * 8), rem = x % ((kN - kHpRow - 1) * 8);
     const int row = kHpRow + 1 + rem / 8, c = rem % 8;
-    tc::st_shared_v4(tc::smem_u32(smem + s * kStageBytes + kWBytes + row * 128 + c * 16), 0u, 0u,
+    tc::st_shared_v4(tc::smem_u32(smem + s * stage_bytes + w_region + row * 128 + c * 16), 0u, 0u,
                      0u, 0u);
   }
   tc::fence_proxy_async();
@@ -124,7 +136,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
       tc::prefetch_tmap(&tm_w);
-      tc::prefetch_tmap(&tm_w16);
       tc::prefetch_tmap(&tm_h);
       tc::prefetch_tmap(&tm_hp);
       const uint64_t pol_w = tc::policy_evict_first();
@@ -140,23 +151,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_arrive(&tile_bar[slot]);  // release: consumers read tile_q after their wait
         if (t < 0) break;
         next = R + atomicAdd(a.tile_ctr, 1);  // the next tile, fetched while this one streams
-        const int vt = t * kVTile, nw = min(kVTile, a.V - vt);
-        const int nbox = nw == kVTile ? 0 : (nw + 15) / 16;
-        const int w_bytes = nbox ? nbox * 2048 : kWBytes;
+        const int vt = t * TR;  // rows past V (last tile) arrive as zeros
         bool ok = true;
         for (int kb = 0; kb < n_k; ++kb) {
           if (!tc::mbar_wait(&empty_bar[s], ph ^ 1, a.status)) { ok = false; break; }
-          uint8_t* st = smem + static_cast<size_t>(s) * kStageBytes;
+          uint8_t* st = smem + static_cast<size_t>(s) * stage_bytes;
           uint64_t* bar = &full_bar[s];
-          // 16 + 16 rows of h and the one row of h_prev
-          tc::mbar_arrive_expect_tx(bar, w_bytes + (2 * 16 + 1) * 128);
-          if (!nbox) tc::tma_load_2d(st, &tm_w, bar, kb * kKStage, vt, pol_w);
-          for (int j = 0; j < nbox; ++j)  // short last tile: accumulator rows past it are ignored
-            tc::tma_load_2d(st + j * 2048, &tm_w16, bar, kb * kKStage, vt + 16 * j, pol_w);
-          tc::tma_load_2d(st + kWBytes, &tm_h, bar, kb * kKStage, 0, pol_h);
-          tc::tma_load_2d(st + kWBytes + 16 * 128, &tm_h, bar, kb * kKStage, 16, pol_h);
-          tc::tma_load_2d(st + kWBytes + kHpRow * 128, &tm_hp, bar, kb * kKStage, 0, pol_h);
-          if (++s == kStages) { s = 0; ph ^= 1; }
+          // TR rows of W, 16 + 16 rows of h and the one row of h_prev
+          tc::mbar_arrive_expect_tx(bar, (TR + 2 * 16 + 1) * 128);
+          tc::tma_load_2d(st, &tm_w, bar, kb * kKStage, vt, pol_w);
+          tc::tma_load_2d(st + w_region, &tm_h, bar, kb * kKStage, 0, pol_h);
+          tc::tma_load_2d(st + w_region + 16 * 128, &tm_h, bar, kb * kKStage, 16, pol_h);
+          tc::tma_load_2d(st + w_region + kHpRow * 128, &tm_hp, bar, kb * kKStage, 0, pol_h);
+          if (++s == n_stages) { s = 0; ph ^= 1; }
         }
         if (!ok) break;
       }
@@ -181,14 +188,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < n_k; ++kb) {
           if (!tc::mbar_wait(&full_bar[s], ph, a.status)) { ok = false; break; }
           tc::tc_fence_after();
-          const uint32_t sa = tc::smem_u32(smem + static_cast<size_t>(s) * kStageBytes);
-          const uint32_t sb = sa + kWBytes;
+          const uint32_t sa = tc::smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+          const uint32_t sb = sa + w_region;
 #pragma unroll
           for (int kk = 0; kk < kKStage / 16; ++kk)
             tc::mma_bf16_ss(d, tc::sdesc_kmajor_sw128(sa + kk * 32),
                             tc::sdesc_kmajor_sw128(sb + kk * 32), idesc, (kb | kk) != 0);
           tc::mma_commit(&empty_bar[s]);
-          if (++s == kStages) { s = 0; ph ^= 1; }
+          if (++s == n_stages) { s = 0; ph ^= 1; }
         }
         tc::mma_commit(&tfull_bar[b]);
       }
@@ -207,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = it & 1;
       if (!tc::mbar_wait_warp(&tfull_bar[b], (it >> 1) & 1, a.status)) break;
       tc::tc_fence_after();
-      const int vbase = t * kVTile + q * 32, vend = min(a.V, t * kVTile + kVTile);
+      const int vbase = t * TR + q * 32, vend = min(a.V, t * TR + TR);
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * 64;
       lmh::fold_chunk(taddr, xpose[q], lane, vbase, vend, run0);       // h[0..31]
       lmh::fold_chunk(taddr + 32, xpose[q], lane, vbase, vend, run1);  // h_prev, unused
@@ -355,11 +362,17 @@ cudaError_t launch_select_fused(int hidden, int vocab, const void* h, const void
                                 int32_t* tokens, uint32_t* unmask, float* pmax_out,
                                 int32_t* argmax_out, float* pm, float* ps, int32_t* pa,
                                 int32_t* header, cudaStream_t st) {
-  CUtensorMap tm_w, tm_w16, tm_h, tm_hp;
+  // Tile rows: the fewest rounds of one tile per CTA that cover the
+  // vocabulary with tiles of at most 128 rows, then the smallest tile size
+  // for that many tiles (at least kMinTileRows).
+  const int R = lmh::sm_count();
+  const long long rounds = (static_cast<long long>(vocab) + static_cast<long long>(R) * kVTile - 1) /
+                           (static_cast<long long>(R) * kVTile);
+  int tr = static_cast<int>((vocab + rounds * R - 1) / (rounds * R));
+  tr = tr < kMinTileRows ? kMinTileRows : (tr > kVTile ? kVTile : tr);
+  CUtensorMap tm_w, tm_h, tm_hp;
   if (!lmh::make_tmap_2d(&tm_w, w, static_cast<uint64_t>(vocab), static_cast<uint64_t>(hidden),
-                         kVTile) ||
-      !lmh::make_tmap_2d(&tm_w16, w, static_cast<uint64_t>(vocab), static_cast<uint64_t>(hidden),
-                         16) ||
+                         static_cast<uint32_t>(tr)) ||
       !lmh::make_tmap_2d(&tm_h, h, kBlock, static_cast<uint64_t>(hidden), 16) ||
       !lmh::make_tmap_2d(&tm_hp, h_prev, 1, static_cast<uint64_t>(hidden), 1))
     return cudaErrorInvalidValue;
@@ -377,13 +390,14 @@ cudaError_t launch_select_fused(int hidden, int vocab, const void* h, const void
   a.ps = ps;
   a.pa = pa;
   a.part_stride = select_fused_part_stride();
+  a.tile_rows = tr;
   a.status = header + 1;
   a.arrivals = reinterpret_cast<uint32_t*>(header + 2);
   a.tile_ctr = header + 3;
   cudaFuncSetAttribute(select_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        kSmemBytes + 1024);
   const cudaError_t e = launch_pdl(select_fused_kernel, dim3(lmh::sm_count()), dim3(kThreads),
-                                   kSmemBytes + 1024, st, tm_w, tm_w16, tm_h, tm_hp, a);
+                                   kSmemBytes + 1024, st, tm_w, tm_h, tm_hp, a);
   if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
