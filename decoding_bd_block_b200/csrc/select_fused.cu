@@ -256,60 +256,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // Partials of the masked positions into shared memory (the ring is idle
-  // now), all loads in flight at once, then one warp per position reduces.
+  // Eight lanes per masked position, each reducing its share of the
+  // position's partials straight from L2 (all its loads in flight at once):
+  // the max and the lowest index attaining it first, then the sum of
+  // exp(m_k - max) s_k, one exponential per part.
   const int P = gridDim.x, PS = a.part_stride;
   const int M = __popc(bits);
   if (warp == 0 && ((bits >> lane) & 1u)) pos_of[__popc(bits & ((1u << lane) - 1u))] = lane;
   __syncthreads();
-  float* lm = reinterpret_cast<float*>(smem);
-  float* ls = lm + kBlock * PS;
-  int* la = reinterpret_cast<int*>(ls + kBlock * PS);
-  {
-    const int vec_per_row = PS / 4;
-    const int total = M * vec_per_row;
-    for (int x0 = threadIdx.x; x0 < total; x0 += kThreads * 8) {
-      uint4 vm[8], vs[8], va[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int x = x0 + u * kThreads;
-        if (x < total) {
-          const int r = x / vec_per_row, c = x % vec_per_row;
-          const size_t g = static_cast<size_t>(pos_of[r]) * PS + 4 * c;
-          vm[u] = __ldcg(reinterpret_cast<const uint4*>(a.pm + g));
-          vs[u] = __ldcg(reinterpret_cast<const uint4*>(a.ps + g));
-          va[u] = __ldcg(reinterpret_cast<const uint4*>(a.pa + g));
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int x = x0 + u * kThreads;
-        if (x < total) {
-          const int r = x / vec_per_row, c = x % vec_per_row;
-          reinterpret_cast<uint4*>(lm + r * PS)[c] = vm[u];
-          reinterpret_cast<uint4*>(ls + r * PS)[c] = vs[u];
-          reinterpret_cast<uint4*>(la + r * PS)[c] = va[u];
-        }
-      }
-    }
-  }
-  __syncthreads();
-  // Eight lanes per position: the max and the lowest index attaining it
-  // first, then the sum of exp(m_k - max) s_k, one exponential per part.
+  constexpr int kVecPerLane = 5;  // 8 lanes x 5 x 4 parts >= part_stride (host-checked)
   for (int r0 = warp * 4; r0 < M; r0 += kThreads / 8) {
     const int r = r0 + lane / 8, j = lane % 8;
     const bool live = r < M;
-    const float* rm = lm + (live ? r : 0) * PS;
-    const float* rs = ls + (live ? r : 0) * PS;
-    const int* ra = la + (live ? r : 0) * PS;
+    const size_t row = static_cast<size_t>(live ? pos_of[r] : 0) * PS;
+    float4 vm[kVecPerLane], vs[kVecPerLane];
+    int4 va[kVecPerLane];
+#pragma unroll
+    for (int u = 0; u < kVecPerLane; ++u) {
+      const int c = j + 8 * u;  // uint4 index within the row
+      vm[u] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      if (live && 4 * c < PS) {
+        vm[u] = __ldcg(reinterpret_cast<const float4*>(a.pm + row) + c);
+        vs[u] = __ldcg(reinterpret_cast<const float4*>(a.ps + row) + c);
+        va[u] = __ldcg(reinterpret_cast<const int4*>(a.pa + row) + c);
+      }
+    }
     float mx = -INFINITY;
     int am = 0x7fffffff;
-    for (int k = j; live && k < P; k += 8) {
-      const float m = rm[k];
-      if (m > mx || (m == mx && ra[k] < am)) {
+    auto take = [&](float m, int ai, int k) {
+      if (k < P && (m > mx || (m == mx && ai < am))) {
         mx = m;
-        am = ra[k];
+        am = ai;
       }
+    };
+#pragma unroll
+    for (int u = 0; u < kVecPerLane; ++u) {
+      const int k = 4 * (j + 8 * u);
+      take(vm[u].x, va[u].x, k);
+      take(vm[u].y, va[u].y, k + 1);
+      take(vm[u].z, va[u].z, k + 2);
+      take(vm[u].w, va[u].w, k + 3);
     }
 #pragma unroll
     for (int o = 4; o > 0; o >>= 1) {
@@ -321,8 +307,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     float sum = 0.f;
-    for (int k = j; live && k < P; k += 8)
-      if (rm[k] != -INFINITY) sum += rs[k] * expf(rm[k] - mx);
+    auto add = [&](float m, float sv, int k) {
+      if (k < P && m != -INFINITY) sum += sv * expf(m - mx);
+    };
+#pragma unroll
+    for (int u = 0; u < kVecPerLane; ++u) {
+      const int k = 4 * (j + 8 * u);
+      add(vm[u].x, vs[u].x, k);
+      add(vm[u].y, vs[u].y, k + 1);
+      add(vm[u].z, vs[u].z, k + 2);
+      add(vm[u].w, vs[u].w, k + 3);
+    }
 #pragma unroll
     for (int o = 4; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     if (live && j == 0) {
@@ -352,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool select_fused_supported(int dtype, int batch, int hidden) {
   return dtype == BD_BF16 && batch == 1 && hidden % 8 == 0 &&
-         kBlock * select_fused_part_stride() * 12 <= kSmemBytes;
+         select_fused_part_stride() <= 8 * 5 * 4;  // the merge's 8 lanes x 5 x float4
 }
 
 int select_fused_part_stride() { return (lmh::sm_count() + 3) / 4 * 4; }
