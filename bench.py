@@ -394,7 +394,8 @@ def run_ours(args, cfg, tau, S, dist: Dist):
 
     e2e = None
     if not args.no_e2e and step.sel:
-        e2e = measure_e2e(step, cfg, tau, S, flush, dev, dist, max(10, K // 4))
+        e2e = measure_e2e(step, cfg, tau, S, flush, dev, dist, max(10, K // 4),
+                          graphs["step"] if graphs else None)
 
     line = {
         "metric": "masked positions scored/s per denoise step",
@@ -425,20 +426,17 @@ def run_ours(args, cfg, tau, S, dist: Dist):
         print(json.dumps(line), flush=True)
 
 
-def measure_e2e(step, cfg, tau, S, flush, dev, dist, K):
+def measure_e2e(step, cfg, tau, S, flush, dev, dist, K, graph=None):
     """Same metric through the public API with the step's inputs on pinned host
-    memory: H2D of the step inputs and D2H of tokens + unmask bits are inside
-    the timed region of every step."""
+    memory: every timed step copies its inputs (q, k_blk, v_blk, h, h_prev,
+    mask bits, tokens: one contiguous host-to-device copy into the step's
+    arena), runs the step (the captured step graph, else eager calls) and
+    reads back the tokens and unmask bits (one device-to-host copy)."""
     import torch
-    host_in = []
-    for name in ("q", "k_blk", "v_blk", "h", "h_prev", "masked", "tokens_in"):
-        t = getattr(step, name, None)
-        if t is not None:
-            host_in.append((t, t.cpu().pin_memory()))
-    tok_h = torch.empty(step.tokens.shape, dtype=step.tokens.dtype).pin_memory()
-    un_h = torch.empty(step.unmask.shape, dtype=step.unmask.dtype).pin_memory()
-    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
-    d2h = tok_h.numel() * tok_h.element_size() + un_h.numel() * un_h.element_size()
+    host_in = step.arena[:step.in_bytes].cpu().pin_memory()
+    host_out = torch.empty(step.arena.numel() - step.out_off, dtype=torch.uint8).pin_memory()
+    h2d = int(host_in.numel())
+    d2h = int(host_out.numel())  # tokens and unmask bits (256-byte aligned within the arena)
     stream = torch.cuda.current_stream(dev)
     times = []
     dist.barrier()
@@ -446,19 +444,20 @@ def measure_e2e(step, cfg, tau, S, flush, dev, dist, K):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for dst, src in host_in:
-            dst.copy_(src, non_blocking=True)
-        step.tokens.copy_(step.tokens_in)
-        step.run(tau, S)
-        tok_h.copy_(step.tokens, non_blocking=True)
-        un_h.copy_(step.unmask, non_blocking=True)
+        step.arena[:step.in_bytes].copy_(host_in, non_blocking=True)
+        if graph is not None:
+            graph.replay()
+        else:
+            step.run(tau, S)
+        host_out.copy_(step.arena[step.out_off:], non_blocking=True)
         e1.record(stream)
         e1.synchronize()
         times.append(e0.elapsed_time(e1))
     ms = dist.max(float(np.mean(times)), dev)
     total = dist.sum(float(step.n_scored), dev)
     return {"value": total / (ms / 1e3), "unit": "masked positions scored/s",
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "launch": "CUDA graph replay" if graph is not None else "eager C-ABI calls"}
 
 
 def run_mask_attn(args, cfg, dist: Dist):

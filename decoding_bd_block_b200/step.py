@@ -47,8 +47,23 @@ class BlockCacheState:
                 bd.bd_cache_commit(self.cache, k, v, [s], nb)
 
 
+def _host_array(a: np.ndarray, dtype: str) -> np.ndarray:
+    """The bytes a tensor of `dtype` holds for array a (bf16 as bit patterns)."""
+    if dtype == "bf16":
+        return np.ascontiguousarray(a).view(np.uint16)
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
 class DecodeStep:
-    """Buffers of one denoising step: block attention + confidence select."""
+    """Buffers of one denoising step: block attention + confidence select.
+
+    The step's per-step inputs (q, k_blk, v_blk, h, h_prev, the mask bits
+    and the block's tokens) and its results (the tokens again and the
+    unmask bits) are views of one device arena, laid out as
+    [inputs ... | tokens | unmask], so that a serving loop moves a step's
+    inputs with one host-to-device copy (``arena[:in_bytes]``) and reads the
+    result back with one device-to-host copy (``arena[out_off:]``).
+    """
 
     def __init__(self, cfg: StepConfig, attn_in: dict | None, sel_in: dict | None,
                  device="cuda", cache: BlockCacheState | None = None):
@@ -56,24 +71,41 @@ class DecodeStep:
         B, dt = cfg.batch, cfg.dtype
         self.attn = attn_in is not None
         self.sel = sel_in is not None
+        tdt = torch_dtype(dt)
+        parts = []  # (name, host array, torch dtype, shape)
+        if self.attn:
+            for name in ("q", "k_blk", "v_blk"):
+                parts.append((name, _host_array(attn_in[name], dt), tdt, attn_in[name].shape))
+        if self.sel:
+            self.masked_host = np.ascontiguousarray(sel_in["masked_bits"], dtype=np.uint32)
+            parts.append(("h", _host_array(sel_in["h"], dt), tdt, sel_in["h"].shape))
+            parts.append(("h_prev", _host_array(sel_in["h_prev"], dt), tdt, sel_in["h_prev"].shape))
+            parts.append(("masked", self.masked_host.view(np.int32), torch.int32, (B,)))
+            parts.append(("tokens", np.ascontiguousarray(sel_in["tokens"], np.int32), torch.int32,
+                          (B, BLOCK)))
+            parts.append(("unmask", np.zeros(B, np.int32), torch.int32, (B,)))
+        offs, off = [], 0
+        for _, arr, _, _ in parts:
+            offs.append(off)
+            off = (off + arr.nbytes + 255) // 256 * 256
+        host = np.zeros(max(off, 256), dtype=np.uint8)
+        for (_, arr, _, _), o in zip(parts, offs):
+            host[o:o + arr.nbytes] = np.frombuffer(arr.tobytes(), dtype=np.uint8)
+        self.arena = torch.from_numpy(host).to(device)
+        for (name, arr, tdtype, shape), o in zip(parts, offs):
+            setattr(self, name, self.arena[o:o + arr.nbytes].view(tdtype).view(*shape))
+        names = [p[0] for p in parts]
+        self.in_bytes = offs[names.index("unmask")] if self.sel else off
+        self.out_off = offs[names.index("tokens")] if self.sel else off
         if self.attn:
             self.cstate = cache or BlockCacheState(cfg, attn_in["prefix_len"], attn_in["prefix_k"],
                                                    attn_in["prefix_v"], device=device)
-            self.q = to_device(attn_in["q"], dt, device)
-            self.k_blk = to_device(attn_in["k_blk"], dt, device)
-            self.v_blk = to_device(attn_in["v_blk"], dt, device)
             self.out = torch.empty_like(self.q)
             n = bd.bd_block_attn_workspace_size(self.cstate.cache)
             self.attn_ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
         if self.sel:
             self.W = to_device(sel_in["W"], dt, device)
-            self.h = to_device(sel_in["h"], dt, device)
-            self.h_prev = to_device(sel_in["h_prev"], dt, device)
-            self.masked_host = np.ascontiguousarray(sel_in["masked_bits"], dtype=np.uint32)
-            self.masked = torch.from_numpy(self.masked_host.view(np.int32)).to(device)
-            self.tokens_in = torch.from_numpy(np.ascontiguousarray(sel_in["tokens"], np.int32)).to(device)
-            self.tokens = self.tokens_in.clone()
-            self.unmask = torch.zeros(B, dtype=torch.int32, device=device)
+            self.tokens_in = self.tokens.clone()
             self.pmax = torch.empty((B, BLOCK), dtype=torch.float32, device=device)
             self.argmax = torch.empty((B, BLOCK), dtype=torch.int32, device=device)
             n = bd.bd_confidence_select_workspace_size(dt, B, cfg.hidden, cfg.vocab)
