@@ -96,6 +96,14 @@ class Dist:
             self.dist.destroy_process_group()
 
 
+def replica_throughput(dist: Dist, units: float, ms_rank: float, device=None):
+    """Whole-job throughput of independent replicas: every rank processed
+    `units` in `ms_rank` ms; the job's time is the slowest rank's.  Returns
+    (ms, units summed over ranks per second)."""
+    ms = dist.max(ms_rank, device)
+    return ms, dist.sum(units, device) / (ms / 1e3)
+
+
 # --------------------------------------------------------------------------
 # clocks sampled during the timed region
 # --------------------------------------------------------------------------
@@ -362,11 +370,9 @@ def run_ours(args, cfg, tau, S, dist: Dist):
     t_sel = [evb[i][1].elapsed_time(evb[i][2]) for i in range(n_bd)]
     t_step = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     ms_rank = float(np.mean(t_step))
-    ms = dist.max(ms_rank, dev)
     n_scored = step.n_scored if step.sel else 0
     unit_count = n_scored if step.sel else cfg.batch * W.BLOCK * cfg.n_heads_q
-    total_units = dist.sum(float(unit_count), dev)
-    value = total_units / (ms / 1e3)
+    ms, value = replica_throughput(dist, float(unit_count), ms_rank, dev)
 
     peaks, peak_kind = measured_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
@@ -453,9 +459,8 @@ def measure_e2e(step, cfg, tau, S, flush, dev, dist, K, graph=None):
         e1.record(stream)
         e1.synchronize()
         times.append(e0.elapsed_time(e1))
-    ms = dist.max(float(np.mean(times)), dev)
-    total = dist.sum(float(step.n_scored), dev)
-    return {"value": total / (ms / 1e3), "unit": "masked positions scored/s",
+    ms, value = replica_throughput(dist, float(step.n_scored), float(np.mean(times)), dev)
+    return {"value": value, "unit": "masked positions scored/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
             "launch": "CUDA graph replay" if graph is not None else "eager C-ABI calls"}
 
@@ -494,16 +499,16 @@ def run_mask_attn(args, cfg, dist: Dist):
     torch.cuda.synchronize(dev)
     dist.barrier()
     launches = bd.bd_kernel_launches() - launches0
-    ms = dist.max(float(np.mean([e[0].elapsed_time(e[1]) for e in ev])), dev)
+    ms, rows_per_s = replica_throughput(dist, float(cfg.n_seqs * 2 * cfg.L * cfg.n_heads_q),
+                                        float(np.mean([e[0].elapsed_time(e[1]) for e in ev])), dev)
     pairs = int(O.mixed_mask(cfg.L, cfg.block).sum())
     flop = 4.0 * cfg.head_dim * cfg.n_heads_q * pairs * cfg.n_seqs
-    rows = dist.sum(float(cfg.n_seqs * 2 * cfg.L * cfg.n_heads_q), dev)
     peaks, peak_kind = measured_peaks()
     peak = float(peaks.get("bf16_tflops", 1590.0))
     ach = flop / (ms / 1e3) / 1e12
     line = {
         "metric": "query rows attended/s (2L x 2L complementary-mask attention)",
-        "value": rows / (ms / 1e3), "unit": "query rows/s", "n_gpus": dist.world, "steps": K,
+        "value": rows_per_s, "unit": "query rows/s", "n_gpus": dist.world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
         "config": {"workload": cfg.name, "views": cfg.n_seqs, "L": cfg.L, "block": cfg.block,
