@@ -22,7 +22,7 @@ STATUS = {0: "BD_OK", -1: "BD_ERR_INVALID_ARG", -2: "BD_ERR_UNSUPPORTED",
 EXPORTED = ("bd_cache_commit", "bd_block_attn_workspace_size", "bd_block_attn",
             "bd_confidence_select_workspace_size", "bd_confidence_select",
             "bd_block_mask_attn", "bd_status_string", "bd_last_cuda_error_string",
-            "bd_kernel_launches", "bd_confidence_select_noalloc")
+            "bd_kernel_launches", "bd_confidence_select_noalloc", "bd_confidence_select_active")
 BD_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 if not os.path.exists(_LIB_PATH):
@@ -69,6 +69,8 @@ _SIGS = {
     "bd_block_mask_attn": [ctypes.POINTER(bd_attn_shape), _P, _P, _P, _P, _I, _I, _I, _P],
     "bd_confidence_select_noalloc": [_I, _I, _I, _I, _P, _P, _P, _P, ctypes.c_float, _I, _P, _P,
                                      _P, _P, _P],
+    "bd_confidence_select_active": [_I, _I, _I, _I, _P, _P, _P, _P, ctypes.c_float, _I, _P, _P,
+                                    _P, _P, _P, ctypes.c_size_t, _P],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -180,6 +182,19 @@ def bd_confidence_select(dtype, batch, hidden, vocab, h, h_prev, w_lm, masked_bi
                          workspace_bytes=None, stream=None):
     wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
     _check("bd_confidence_select", _lib.bd_confidence_select(
+        dtype_code(dtype), int(batch), int(hidden), int(vocab), _ptr(h), _ptr(h_prev),
+        _ptr(w_lm), _ptr(masked_bits), float(tau), int(sub_block), _ptr(tokens),
+        _ptr(unmask_bits), _ptr(pmax_out), _ptr(argmax_out), _ptr(workspace), int(wsb),
+        _stream(stream)))
+
+
+def bd_confidence_select_active(dtype, batch, hidden, vocab, h, h_prev, w_lm, masked_bits, tau,
+                                sub_block, tokens, unmask_bits, pmax_out, argmax_out, workspace,
+                                workspace_bytes=None, stream=None):
+    """bd_confidence_select scoring only the unmask rule's candidates (the
+    masked positions of the lowest sub-block that has one; see include/bd.h)."""
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check("bd_confidence_select_active", _lib.bd_confidence_select_active(
         dtype_code(dtype), int(batch), int(hidden), int(vocab), _ptr(h), _ptr(h_prev),
         _ptr(w_lm), _ptr(masked_bits), float(tau), int(sub_block), _ptr(tokens),
         _ptr(unmask_bits), _ptr(pmax_out), _ptr(argmax_out), _ptr(workspace), int(wsb),

@@ -164,11 +164,11 @@ int bd_confidence_select_workspace_size(int32_t dtype, int32_t batch, int32_t hi
   return BD_OK;
 }
 
-int bd_confidence_select(int32_t dtype, int32_t batch, int32_t hidden, int32_t vocab,
-                         const void* h, const void* h_prev, const void* w,
-                         const uint32_t* masked_bits, float tau, int32_t sub_block,
-                         int32_t* tokens, uint32_t* unmask_bits, float* pmax_out,
-                         int32_t* argmax_out, void* ws, size_t ws_bytes, void* stream) {
+namespace {
+int confidence_select(int32_t dtype, int32_t batch, int32_t hidden, int32_t vocab, const void* h,
+                      const void* h_prev, const void* w, const uint32_t* masked_bits, float tau,
+                      int32_t sub_block, int32_t* tokens, uint32_t* unmask_bits, float* pmax_out,
+                      int32_t* argmax_out, void* ws, size_t ws_bytes, void* stream, int active) {
   if (batch <= 0 || batch > 65535 || hidden <= 0 || vocab <= 0) return BD_ERR_INVALID_ARG;
   if (dtype != BD_F32 && dtype != BD_BF16) return BD_ERR_UNSUPPORTED;
   if (hidden % 8 != 0) return BD_ERR_UNSUPPORTED;
@@ -186,7 +186,26 @@ int bd_confidence_select(int32_t dtype, int32_t batch, int32_t hidden, int32_t v
   return cuda_status(bd::launch_confidence_select(dtype, batch, hidden, vocab, p, h, h_prev, w,
                                                   masked_bits, tau, sub_block, tokens,
                                                   unmask_bits, pmax_out, argmax_out, ws,
-                                                  static_cast<cudaStream_t>(stream)));
+                                                  static_cast<cudaStream_t>(stream), active));
+}
+}  // namespace
+
+int bd_confidence_select(int32_t dtype, int32_t batch, int32_t hidden, int32_t vocab,
+                         const void* h, const void* h_prev, const void* w,
+                         const uint32_t* masked_bits, float tau, int32_t sub_block,
+                         int32_t* tokens, uint32_t* unmask_bits, float* pmax_out,
+                         int32_t* argmax_out, void* ws, size_t ws_bytes, void* stream) {
+  return confidence_select(dtype, batch, hidden, vocab, h, h_prev, w, masked_bits, tau, sub_block,
+                           tokens, unmask_bits, pmax_out, argmax_out, ws, ws_bytes, stream, 0);
+}
+
+int bd_confidence_select_active(int32_t dtype, int32_t batch, int32_t hidden, int32_t vocab,
+                                const void* h, const void* h_prev, const void* w,
+                                const uint32_t* masked_bits, float tau, int32_t sub_block,
+                                int32_t* tokens, uint32_t* unmask_bits, float* pmax_out,
+                                int32_t* argmax_out, void* ws, size_t ws_bytes, void* stream) {
+  return confidence_select(dtype, batch, hidden, vocab, h, h_prev, w, masked_bits, tau, sub_block,
+                           tokens, unmask_bits, pmax_out, argmax_out, ws, ws_bytes, stream, 1);
 }
 
 int bd_block_mask_attn(const bd_attn_shape* sh, const void* q, const void* k, const void* v,

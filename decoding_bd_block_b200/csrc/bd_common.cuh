@@ -158,6 +158,16 @@ __device__ __forceinline__ void select_sequence(int s, uint32_t bits, float p, i
   if (argmax_out) argmax_out[s * kBlock + i] = is_m ? tok : -1;
 }
 
+// The positions one step scores: every masked position, or -- active-only
+// scoring -- the masked positions of the lowest sub-block of S positions
+// that still has one, the only candidates the unmask rule can pick.
+__device__ __forceinline__ uint32_t scored_bits(uint32_t bits, int S, int active) {
+  if (!active || !bits) return bits;
+  const int k0 = ((__ffs(static_cast<int>(bits)) - 1) / S) * S;
+  const uint32_t win = S >= 32 ? 0xffffffffu : ((1u << S) - 1u) << k0;
+  return bits & win;
+}
+
 // "No decision" for sequence s (a bounded wait gave up): nothing is
 // unmasked, p_max is NaN and the token -2.  Lane i of one warp writes position i.
 __device__ __forceinline__ void no_decision_sequence(int s, uint32_t* unmask, float* pmax_out,
@@ -236,8 +246,8 @@ cudaError_t launch_block_attn(const bd_attn_shape& sh, const bd_kv_cache& c, con
 // The packed-row count is the popcount of masked[0 .. batch).
 int lmhead_tc_grid();
 cudaError_t launch_lmhead_tc(const void* rows, const void* w, const uint32_t* masked, int batch,
-                             int H, int V, int rows_alloc, int part_stride, float* pm, float* ps,
-                             int32_t* pa, int32_t* status, cudaStream_t st);
+                             int S, int active, int H, int V, int rows_alloc, int part_stride,
+                             float* pm, float* ps, int32_t* pa, int32_t* status, cudaStream_t st);
 
 struct SelectPlan {
   bool fused;        // one kernel, rows resident in shared memory (select_fused.cu)
@@ -257,13 +267,15 @@ cudaError_t launch_select_fused(int hidden, int vocab, const void* h, const void
                                 const void* w, const uint32_t* masked, float tau, int sub_block,
                                 int32_t* tokens, uint32_t* unmask, float* pmax_out,
                                 int32_t* argmax_out, float* pm, float* ps, int32_t* pa,
-                                int32_t* header, cudaStream_t st);
+                                int32_t* header, int active, cudaStream_t st);
+// active != 0: score only the active sub-block's masked positions (see
+// scored_bits); the decisions are the same, p_max / argmax elsewhere NaN / -1.
 cudaError_t launch_confidence_select(int dtype, int batch, int hidden, int vocab,
                                      const SelectPlan& p, const void* h, const void* h_prev,
                                      const void* w, const uint32_t* masked, float tau,
                                      int sub_block, int32_t* tokens, uint32_t* unmask,
                                      float* pmax_out, int32_t* argmax_out, void* ws,
-                                     cudaStream_t st);
+                                     cudaStream_t st, int active = 0);
 
 // Tensor-core mask attention (mask_attn_tc.cu): bf16, head_dim 128, L % 128 == 0.
 bool mask_attn_tc_supported(const bd_attn_shape& sh, int L);

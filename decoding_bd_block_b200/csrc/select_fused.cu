@@ -53,6 +53,7 @@ __host__ __device__ constexpr int stage_w_bytes(int tr) {
 
 struct FusedArgs {
   const uint32_t* masked;  // [1]
+  int active;              // score only the active sub-block (scored_bits)
   int H, V;
   float tau;
   int S;
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = tmem_slot;
   griddep_wait();  // first kernel of the call: the caller's inputs are complete after this
   griddep_launch_dependents();
-  const uint32_t bits = a.masked[0];
+  const uint32_t bits = scored_bits(a.masked[0], a.S, a.active);
 
   if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
@@ -356,7 +357,7 @@ cudaError_t launch_select_fused(int hidden, int vocab, const void* h, const void
                                 const void* w, const uint32_t* masked, float tau, int sub_block,
                                 int32_t* tokens, uint32_t* unmask, float* pmax_out,
                                 int32_t* argmax_out, float* pm, float* ps, int32_t* pa,
-                                int32_t* header, cudaStream_t st) {
+                                int32_t* header, int active, cudaStream_t st) {
   // Tile rows: the fewest rounds of one tile per CTA that cover the
   // vocabulary with tiles of at most 128 rows, then the smallest tile size
   // for that many tiles (at least kMinTileRows).
@@ -373,6 +374,7 @@ cudaError_t launch_select_fused(int hidden, int vocab, const void* h, const void
     return cudaErrorInvalidValue;
   FusedArgs a{};
   a.masked = masked;
+  a.active = active;
   a.H = hidden;
   a.V = vocab;
   a.tau = tau;

@@ -24,14 +24,14 @@ template <typename T>
 __global__ void __launch_bounds__(1024) gather_rows_kernel(
     const T* __restrict__ h, const T* __restrict__ h_prev, const uint32_t* __restrict__ masked,
     int B, int H, T* __restrict__ rows, int32_t* __restrict__ posrow,
-    int32_t* __restrict__ count, int rows_alloc) {
+    int32_t* __restrict__ count, int rows_alloc, int S, int active) {
   __shared__ int red[32];
   griddep_wait();  // first kernel of the call: the caller's inputs are complete after this
   griddep_launch_dependents();
   const int s = blockIdx.x;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   int acc = 0;
-  for (int x = threadIdx.x; x < s; x += blockDim.x) acc += __popc(masked[x]);
+  for (int x = threadIdx.x; x < s; x += blockDim.x) acc += __popc(scored_bits(masked[x], S, active));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (lane == 0) red[warp] = acc;
@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(1024) gather_rows_kernel(
   int off = 0;
 #pragma unroll
   for (int w = 0; w < 32; ++w) off += red[w];
-  const uint32_t bits = masked[s];
+  const uint32_t bits = scored_bits(masked[s], S, active);
   const int i = warp;
   const bool is_m = (bits >> i) & 1u;
   const int r = is_m ? off + __popc(bits & ((1u << i) - 1u)) : -1;
@@ -148,14 +148,14 @@ __global__ void __launch_bounds__(1024) merge_select_kernel(
     const uint32_t* __restrict__ masked, int n_split, int grouped, const float* __restrict__ pm,
     const float* __restrict__ ps, const int32_t* __restrict__ pa, float tau, int S,
     int32_t* __restrict__ tokens, uint32_t* __restrict__ unmask, float* __restrict__ pmax_out,
-    int32_t* __restrict__ argmax_out) {
+    int32_t* __restrict__ argmax_out, int active) {
   __shared__ float sp[kBlock];
   __shared__ int stok[kBlock];
   griddep_wait();  // the LM head's partials
   griddep_launch_dependents();
   const int s = blockIdx.x;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const uint32_t bits = masked[s];
+  const uint32_t bits = scored_bits(masked[s], S, active);
   if (count[1] != 0) {
     if (warp == 0) no_decision_sequence(s, unmask, pmax_out, argmax_out);
     return;
@@ -236,7 +236,7 @@ static cudaError_t launch_select_t(int batch, int hidden, int vocab, const Selec
                                    const void* h, const void* h_prev, const void* w,
                                    const uint32_t* masked, float tau, int S, int32_t* tokens,
                                    uint32_t* unmask, float* pmax_out, int32_t* argmax_out,
-                                   void* ws, cudaStream_t st) {
+                                   void* ws, cudaStream_t st, int active) {
   char* base = static_cast<char*>(ws);
   T* rows = reinterpret_cast<T*>(base + p.off_rows);
   int32_t* posrow = reinterpret_cast<int32_t*>(base + p.off_posrow);
@@ -246,15 +246,15 @@ static cudaError_t launch_select_t(int batch, int hidden, int vocab, const Selec
   int32_t* pa = reinterpret_cast<int32_t*>(base + p.off_pa);
   if (p.fused)
     return launch_select_fused(hidden, vocab, h, h_prev, w, masked, tau, S, tokens, unmask,
-                               pmax_out, argmax_out, pm, ps, pa, count, st);
+                               pmax_out, argmax_out, pm, ps, pa, count, active, st);
   cudaError_t e = launch_pdl(gather_rows_kernel<T>, dim3(batch), dim3(1024), 0, st,
                              static_cast<const T*>(h), static_cast<const T*>(h_prev), masked,
-                             batch, hidden, rows, posrow, count, p.rows_alloc);
+                             batch, hidden, rows, posrow, count, p.rows_alloc, S, active);
   if (e != cudaSuccess) return e;
   count_launches(1);
   if (p.tc) {
-    e = launch_lmhead_tc(rows, w, masked, batch, hidden, vocab, p.rows_alloc, p.n_split, pm, ps,
-                         pa, count + 1, st);
+    e = launch_lmhead_tc(rows, w, masked, batch, S, active, hidden, vocab, p.rows_alloc,
+                         p.n_split, pm, ps, pa, count + 1, st);
     if (e != cudaSuccess) return e;
   } else {
     lmhead_simt_kernel<T><<<dim3(p.n_split, p.rows_alloc / 32), 256, 0, st>>>(
@@ -264,7 +264,8 @@ static cudaError_t launch_select_t(int batch, int hidden, int vocab, const Selec
   e = launch_pdl(merge_select_kernel, dim3(batch), dim3(1024), 0, st, posrow,
                  static_cast<const int32_t*>(count), masked, p.n_split, p.tc ? 1 : 0,
                  static_cast<const float*>(pm), static_cast<const float*>(ps),
-                 static_cast<const int32_t*>(pa), tau, S, tokens, unmask, pmax_out, argmax_out);
+                 static_cast<const int32_t*>(pa), tau, S, tokens, unmask, pmax_out, argmax_out,
+                 active);
   if (e != cudaSuccess) return e;
   count_launches(1);
   return cudaGetLastError();
@@ -275,12 +276,12 @@ cudaError_t launch_confidence_select(int dtype, int batch, int hidden, int vocab
                                      const void* w, const uint32_t* masked, float tau,
                                      int sub_block, int32_t* tokens, uint32_t* unmask,
                                      float* pmax_out, int32_t* argmax_out, void* ws,
-                                     cudaStream_t st) {
+                                     cudaStream_t st, int active) {
   if (dtype == BD_BF16)
     return launch_select_t<bf16>(batch, hidden, vocab, p, h, h_prev, w, masked, tau, sub_block,
-                                 tokens, unmask, pmax_out, argmax_out, ws, st);
+                                 tokens, unmask, pmax_out, argmax_out, ws, st, active);
   return launch_select_t<float>(batch, hidden, vocab, p, h, h_prev, w, masked, tau, sub_block,
-                                tokens, unmask, pmax_out, argmax_out, ws, st);
+                                tokens, unmask, pmax_out, argmax_out, ws, st, active);
 }
 
 }  // namespace bd

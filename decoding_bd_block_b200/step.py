@@ -71,6 +71,7 @@ class DecodeStep:
         B, dt = cfg.batch, cfg.dtype
         self.attn = attn_in is not None
         self.sel = sel_in is not None
+        self.active_only = False  # score only the unmask rule's candidates
         tdt = torch_dtype(dt)
         parts = []  # (name, host array, torch dtype, shape)
         if self.attn:
@@ -116,20 +117,25 @@ class DecodeStep:
         bd.bd_block_attn(self.cstate.cache, self.q, self.k_blk, self.v_blk, self.out,
                          self.attn_ws, stream=stream)
 
-    def run_select(self, tau: float, sub_block: int, stream=None, outputs=True):
+    def run_select(self, tau: float, sub_block: int, stream=None, outputs=True,
+                   active_only=None):
+        """active_only (default: the step's `active_only`) scores only the
+        unmask rule's candidates (bd_confidence_select_active)."""
         cfg = self.cfg
-        bd.bd_confidence_select(cfg.dtype, cfg.batch, cfg.hidden, cfg.vocab, self.h, self.h_prev,
-                                self.W, self.masked, tau, sub_block, self.tokens, self.unmask,
-                                self.pmax if outputs else None, self.argmax if outputs else None,
-                                self.sel_ws, stream=stream)
+        if active_only is None:
+            active_only = self.active_only
+        fn = bd.bd_confidence_select_active if active_only else bd.bd_confidence_select
+        fn(cfg.dtype, cfg.batch, cfg.hidden, cfg.vocab, self.h, self.h_prev, self.W, self.masked,
+           tau, sub_block, self.tokens, self.unmask, self.pmax if outputs else None,
+           self.argmax if outputs else None, self.sel_ws, stream=stream)
 
-    def run(self, tau: float, sub_block: int, stream=None):
+    def run(self, tau: float, sub_block: int, stream=None, active_only=None):
         if self.attn:
             self.run_attn(stream)
         if self.sel:
-            self.run_select(tau, sub_block, stream)
+            self.run_select(tau, sub_block, stream, active_only=active_only)
 
-    def capture(self, tau: float, sub_block: int, parts=("attn", "select")):
+    def capture(self, tau: float, sub_block: int, parts=("attn", "select"), active_only=None):
         """Record the step's launches (the same C-ABI calls) into CUDA graphs.
 
         Returns {part: torch.cuda.CUDAGraph}; replaying a graph re-runs that
@@ -143,7 +149,7 @@ class DecodeStep:
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
-            self.run(tau, sub_block)          # warm the launch path outside capture
+            self.run(tau, sub_block, active_only=active_only)  # warm the launch path outside capture
         torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
         for part in parts:
@@ -154,9 +160,9 @@ class DecodeStep:
                 if part == "attn":
                     self.run_attn(side)
                 elif part == "select":
-                    self.run_select(tau, sub_block, side)
+                    self.run_select(tau, sub_block, side, active_only=active_only)
                 else:
-                    self.run(tau, sub_block, side)
+                    self.run(tau, sub_block, side, active_only=active_only)
             graphs[part] = g
         torch.cuda.synchronize()
         return graphs

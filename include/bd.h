@@ -180,6 +180,25 @@ BD_API int bd_confidence_select(int32_t dtype, int32_t batch, int32_t hidden,
                          int32_t* argmax_out, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* bd_confidence_select_active -- bd_confidence_select that scores only the
+ * candidates of the unmask rule.
+ *
+ * The rule picks only among the masked positions of the lowest sub-block
+ * that still has one ([N1] key design 4: the sub-block sets the decoding
+ * granularity inside the block), so scoring the other masked positions
+ * decides nothing.  This call computes the LM-head statistics for those
+ * candidates alone (at most sub_block positions per sequence instead of up
+ * to 32).  Same arguments, workspace and errors as bd_confidence_select;
+ * tokens and unmask_bits are the same; pmax_out / argmax_out hold NaN / -1
+ * at every position that is not a candidate. */
+BD_API int bd_confidence_select_active(int32_t dtype, int32_t batch, int32_t hidden,
+                                int32_t vocab, const void* h, const void* h_prev,
+                                const void* w_lm, const uint32_t* masked_bits,
+                                float tau, int32_t sub_block, int32_t* tokens,
+                                uint32_t* unmask_bits, float* pmax_out,
+                                int32_t* argmax_out, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
 /* bd_confidence_select_noalloc -- bd_confidence_select without a workspace.
  *
  * The method's description has no counterpart to this call: it exists for

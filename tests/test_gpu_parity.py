@@ -220,6 +220,36 @@ def test_confidence_select_parity(case):
             assert bin(int(step.unmask[b].item()) & 0xFFFFFFFF).count("1") == want
 
 
+ACTIVE_CASES = [
+    (W.TINY_F32, 0.9, 8),                                     # fp32, CUDA-core LM head
+    (W.QWEN15B_STEP, 0.9, 8),                                 # batch 1: the single kernel
+    (W.QWEN7B_RAGGED, 0.9, 8),                                # tensor-core LM head, packed rows
+    (dataclasses.replace(W.QWEN15B_STEP, name="bf16_b5_active", vocab=1000, hidden=512, batch=5,
+                         n_masked=0, masked_range=(0, 32), seed=105), 0.5, 4),
+    (dataclasses.replace(W.QWEN15B_STEP, name="bf16_b1_s32_active", vocab=3000, hidden=512,
+                         n_masked=30, seed=106), 0.9, 32),
+]
+
+
+@pytest.mark.parametrize("case", ACTIVE_CASES, ids=lambda c: f"{c[0].name}-tau{c[1]}-S{c[2]}")
+def test_confidence_select_active_parity(case):
+    """Scoring only the unmask rule's candidates: the same tokens and unmask
+    bits as the full oracle step; p_max / argmax at the candidates only."""
+    from decoding_bd_block_b200 import bd
+    cfg, tau, S = case
+    _, s, step = _step(cfg, attn=False)
+    n0 = bd.bd_kernel_launches()
+    step.run_select(tau, S, active_only=True)
+    torch.cuda.synchronize()
+    ref = O.confidence_select(s["h"], s["h_prev"], s["W"], s["masked_bits"], tau, S,
+                              s["tokens"], cfg.dtype)
+    cand = np.array([sum(1 << i for i in O.active_candidates(int(b), S)) for b in s["masked_bits"]],
+                    dtype=np.uint32)
+    res = compare_select(ref, step.tokens.cpu().numpy(), step.unmask.cpu().numpy().view(np.uint32),
+                         step.pmax.cpu().numpy(), step.argmax.cpu().numpy(), cand)
+    print(cfg.name, tau, S, res, "launches", bd.bd_kernel_launches() - n0)
+
+
 @pytest.mark.parametrize("batch", [1, 3])  # single-kernel and three-kernel paths
 def test_select_idempotent_and_masked_untouched(batch):
     cfg = dataclasses.replace(W.QWEN15B_STEP, batch=batch, vocab=4096, seed=99)
