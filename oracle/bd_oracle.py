@@ -46,6 +46,13 @@ R7  Selection ([N1] key designs 3 and 4; [N2] item 2; [N4] item 2):
     single c with the largest p_max, ties to the lowest position.  The strict
     comparison is the one under which tau = 1.0 reduces to one token per step
     ([N1] key design 3).  Every masked position of the block is scored.
+R9  Masked-token cross-entropy of training ([N1] key design 2, the L_block
+    equation with the shifted label): in every training sequence (the noisy
+    stream x_t, L positions), each position i >= 1 whose token is [MASK]
+    contributes -log softmax(W h_{i-1})[x_0^i]; position 0 has no previous
+    row in its sequence and contributes nothing.  The equation's
+    expectation is left to the caller: the step returns the per-position
+    losses and their sum over the scored positions.
 R8  Ambiguity: a position's token is ambiguous when its top-2 logit gap is
     < 1e-3; a sequence's unmask decision is ambiguous when some candidate has
     |p_max - tau| < 1e-4 (only for tau < 1: p_max = 1/Z with Z >= 1 never
@@ -68,7 +75,7 @@ __all__ = [
     "block_causal_allowed", "OracleCache", "block_attn_seq", "block_attn",
     "full_sequence_attn", "mixed_mask", "mask_attn", "shifted_rows",
     "lm_logits", "softmax_stats", "active_candidates", "select",
-    "ambiguity", "confidence_select",
+    "ambiguity", "confidence_select", "ce_positions", "masked_ce",
 ]
 
 
@@ -362,3 +369,41 @@ def confidence_select(h, h_prev, W, masked_bits, tau: float, sub_block: int, tok
     return dict(pmax=pmax, argmax=arg, gap=gap, tokens=tok, unmask=unmask,
                 token_ambiguous=tok_amb, decision_ambiguous=dec_amb,
                 n_scored=len(where))
+
+
+# ----------------------------------------------------------------------------
+# masked-token cross-entropy of training (reading R9)
+# ----------------------------------------------------------------------------
+def ce_positions(masked_bits):
+    """Scored positions (sequence, i): [MASK] in x_t and i >= 1, in order.
+
+    masked_bits ``[S, L/32]``: bit i % 32 of word i // 32 marks position i.
+    """
+    bits = np.asarray(masked_bits)
+    S, nw = bits.shape
+    return [(s, i) for s in range(S) for i in range(1, nw * 32)
+            if (int(bits[s, i // 32]) >> (i % 32)) & 1]
+
+
+def masked_ce(h, W, targets, masked_bits, dtype: str = "f32", positions=None, chunk: int = 256):
+    """-log softmax(W h_{i-1})[targets_i] at every scored position (R9).
+
+    h ``[S, L, H]``, W ``[V, H]`` (fp32 arrays or bf16 bit patterns per
+    ``dtype``), targets ``[S, L]``, masked_bits ``[S, L/32]``.  ``positions``
+    restricts the work to a subset of the scored positions (large cases).
+    Returns dict(loss ``[S, L]`` with NaN where not computed, total = sum of
+    the computed losses, count).
+    """
+    S, L = np.asarray(targets).shape
+    pos = ce_positions(masked_bits) if positions is None else list(positions)
+    loss = np.full((S, L), np.nan)
+    for c0 in range(0, len(pos), chunk):
+        part = pos[c0:c0 + chunk]
+        rows = np.stack([widen(h[s, i - 1], dtype) for s, i in part]).astype(np.float64)
+        logits = lm_logits(rows, W, dtype)
+        top = logits.max(axis=1)
+        lse = top + np.log(np.exp(logits - top[:, None]).sum(axis=1))
+        for r, (s, i) in enumerate(part):
+            loss[s, i] = lse[r] - logits[r, int(targets[s, i])]
+    vals = np.array([loss[s, i] for s, i in pos], dtype=np.float64)
+    return dict(loss=loss, total=float(vals.sum()), count=len(pos))

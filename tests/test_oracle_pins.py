@@ -358,3 +358,81 @@ def test_ambiguity_flags():
     p1[1, :2] = [0.99999, 0.999991]
     _, dec1 = O.ambiguity(p1, np.ones((2, 32)), np.array([0b11, 0b11], np.uint32), 1.0, 8)
     np.testing.assert_array_equal(dec1, [False, True])
+
+
+# ------------------------------------------------ masked cross-entropy (R9)
+def _ce_case(S=2, L=64, H=8, V=11, seed=3, frac=0.5):
+    r = np.random.default_rng(seed)
+    h = r.standard_normal((S, L, H)).astype(np.float32)
+    W = r.standard_normal((V, H)).astype(np.float32)
+    y = r.integers(0, V, (S, L)).astype(np.int32)
+    m = r.random((S, L)) < frac
+    m[:, 0] = True  # position 0 is masked but has no previous row
+    bits = np.zeros((S, L // 32), np.uint32)
+    for s in range(S):
+        for i in range(L):
+            if m[s, i]:
+                bits[s, i // 32] |= np.uint32(1 << (i % 32))
+    return h, W, y, bits, m
+
+
+def test_ce_uniform_logits_give_log_vocab():
+    h, W, y, bits, m = _ce_case()
+    out = O.masked_ce(h, np.zeros_like(W), y, bits)
+    scored = m.copy()
+    scored[:, 0] = False
+    assert out["count"] == int(scored.sum())
+    assert np.allclose(out["loss"][scored], math.log(W.shape[0]), rtol=0, atol=1e-14)
+    assert np.isnan(out["loss"][~scored]).all()          # position 0 and unmasked: nothing
+    assert out["total"] == pytest.approx(out["count"] * math.log(W.shape[0]), rel=1e-14)
+
+
+def test_ce_closed_form_one_hot_logits():
+    # W[v] = e_v, h_{i-1} = c e_t: the logits are c at t and 0 elsewhere, so
+    # the loss is log(1 + (V-1) e^-c) when the target is t, log(e^c + V - 1) - 0 otherwise.
+    V, c = 5, 3.0
+    W = np.eye(V, dtype=np.float32)
+    h = np.zeros((1, 32, V), np.float32)
+    t = [(i * 3) % V for i in range(32)]
+    for i in range(32):
+        h[0, i, t[i]] = c
+    y = np.array([[t[i - 1] if i % 2 else (t[i - 1] + 1) % V for i in range(32)]], np.int32)
+    bits = np.array([[0xFFFFFFFE]], np.uint32)
+    out = O.masked_ce(h, W, y, bits)
+    for i in range(1, 32):
+        want = (math.log(1 + (V - 1) * math.exp(-c)) if i % 2
+                else math.log(math.exp(c) + V - 1))
+        assert out["loss"][0, i] == pytest.approx(want, rel=1e-14)
+
+
+def test_ce_matches_library_cross_entropy_with_shift():
+    torch = pytest.importorskip("torch")
+    h, W, y, bits, m = _ce_case(S=3, L=96, H=16, V=37, seed=11)
+    out = O.masked_ce(h, W, y, bits)
+    for s in range(3):
+        idx = [i for i in range(1, 96) if m[s, i]]
+        logits = torch.from_numpy(h[s, [i - 1 for i in idx]].astype(np.float64)) @ \
+            torch.from_numpy(W.astype(np.float64)).T
+        ref = torch.nn.functional.cross_entropy(logits, torch.from_numpy(y[s, idx]).long(),
+                                                reduction="none").numpy()
+        assert np.allclose(out["loss"][s, idx], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_ce_reads_the_previous_row_only():
+    h, W, y, bits, m = _ce_case(S=1, L=64, seed=5, frac=1.0)
+    base = O.masked_ce(h, W, y, bits)["loss"]
+    h2 = h.copy()
+    h2[0, 10] += 1.0                      # row 10 predicts position 11 only
+    out = O.masked_ce(h2, W, y, bits)["loss"]
+    changed = np.nonzero(~np.isclose(out[0], base[0], equal_nan=True))[0].tolist()
+    assert changed == [11]
+
+
+def test_ce_subset_positions_match_full():
+    h, W, y, bits, m = _ce_case(S=2, L=64, seed=9)
+    full = O.masked_ce(h, W, y, bits)
+    pos = O.ce_positions(bits)[::3]
+    part = O.masked_ce(h, W, y, bits, positions=pos)
+    for s, i in pos:
+        assert part["loss"][s, i] == full["loss"][s, i]
+    assert part["count"] == len(pos)
