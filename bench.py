@@ -46,7 +46,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=sorted(W.STEP_CONFIGS) + [W.MASK_ATTN.name])
+                    choices=sorted(W.STEP_CONFIGS) + [W.MASK_ATTN.name, W.MASKED_CE.name])
     ap.add_argument("--tau", type=float, default=None)
     ap.add_argument("--sub-block", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
@@ -483,11 +483,19 @@ def measure_e2e(step, cfg, tau, S, flush, dev, dist, K, graph=None):
             "launch": "CUDA graph replay" if graph is not None else "eager C-ABI calls"}
 
 
+def mask_pairs(L: int, D: int) -> int:
+    """Allowed (query, key) pairs of the 2L x 2L training mask, per view and
+    head: a noisy query of block b sees its own block's D noisy keys and the
+    b D clean keys before it; a clean query of block b sees (b + 1) D clean
+    keys.  Summed over the n = L / D blocks: D^2 (n^2 + n)."""
+    n = L // D
+    return D * D * (n * n + n)
+
+
 def run_mask_attn(args, cfg, dist: Dist):
     """bd_block_mask_attn on the training-forward workload (2L x 2L mask)."""
     import torch
 
-    import oracle as O
     from decoding_bd_block_b200 import bd
     from decoding_bd_block_b200.step import to_device
 
@@ -519,7 +527,7 @@ def run_mask_attn(args, cfg, dist: Dist):
     launches = bd.bd_kernel_launches() - launches0
     ms, rows_per_s = replica_throughput(dist, float(cfg.n_seqs * 2 * cfg.L * cfg.n_heads_q),
                                         float(np.mean([e[0].elapsed_time(e[1]) for e in ev])), dev)
-    pairs = int(O.mixed_mask(cfg.L, cfg.block).sum())
+    pairs = mask_pairs(cfg.L, cfg.block)
     flop = 4.0 * cfg.head_dim * cfg.n_heads_q * pairs * cfg.n_seqs
     peaks, peak_kind = measured_peaks()
     peak = float(peaks.get("bf16_tflops", 1590.0))
@@ -543,6 +551,73 @@ def run_mask_attn(args, cfg, dist: Dist):
         print(json.dumps(line), flush=True)
 
 
+def run_masked_ce(args, cfg, dist: Dist):
+    """bd_masked_ce on the training batch (16 sequences of 2048 positions)."""
+    import torch
+
+    from decoding_bd_block_b200 import bd
+    from decoding_bd_block_b200.step import to_device
+
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    d = W.make_ce_inputs(cfg)
+    N, L = d["targets"].shape
+    h = to_device(d["h"], cfg.dtype, dev)
+    w = to_device(d["W"], cfg.dtype, dev)
+    tg = torch.from_numpy(d["targets"]).to(dev)
+    mb = torch.from_numpy(d["masked_bits"].view(np.int32)).to(dev)
+    loss = torch.empty((N, L), dtype=torch.float32, device=dev)
+    ls = torch.zeros(1, dtype=torch.float32, device=dev)
+    ns = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = torch.empty(bd.bd_masked_ce_workspace_size(cfg.dtype, N, L, cfg.hidden, cfg.vocab),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call = lambda: bd.bd_masked_ce(cfg.dtype, N, L, cfg.hidden, cfg.vocab, h, w, tg, mb, loss, ls,
+                                   ns, ws)
+    for _ in range(args.warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize(dev)
+    count = int(ns.item())
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    launches0 = bd.bd_kernel_launches()
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        call()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    launches = bd.bd_kernel_launches() - launches0
+    ms, value = replica_throughput(dist, float(count),
+                                   float(np.mean([e[0].elapsed_time(e[1]) for e in ev])), dev)
+    flop = 2.0 * count * cfg.vocab * cfg.hidden
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    ach = flop / (ms / 1e3) / 1e12
+    line = {
+        "metric": "masked positions' cross-entropy computed/s (training batch)",
+        "value": value, "unit": "scored positions/s", "n_gpus": dist.world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "config": {"workload": cfg.name, "sequences": N, "L": L, "hidden": cfg.hidden,
+                   "vocab": cfg.vocab, "scored_positions": count,
+                   "mean_loss": float(ls.item()) / max(count, 1),
+                   "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)"},
+        "roofline": {"kernel": "bd_masked_ce (LM head on tcgen05; whole call timed)",
+                     "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                     "frac": ach / peak, "traffic": recorded_traffic("masked_ce"),
+                     "algorithmic_flop_per_launch": flop, "peak_source": peak_kind},
+        "gpu_launches": int(launches),
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.workload == W.MASK_ATTN.name:
@@ -553,6 +628,17 @@ def main(argv=None):
         dist = Dist("nccl")
         try:
             run_mask_attn(args, W.MASK_ATTN, dist)
+        finally:
+            dist.close()
+        return 0
+    if args.workload == W.MASKED_CE.name:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the reference arm times the decoding-step workloads only"}))
+            return 0
+        dist = Dist("nccl")
+        try:
+            run_masked_ce(args, W.MASKED_CE, dist)
         finally:
             dist.close()
         return 0

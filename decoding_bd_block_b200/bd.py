@@ -22,7 +22,8 @@ STATUS = {0: "BD_OK", -1: "BD_ERR_INVALID_ARG", -2: "BD_ERR_UNSUPPORTED",
 EXPORTED = ("bd_cache_commit", "bd_block_attn_workspace_size", "bd_block_attn",
             "bd_confidence_select_workspace_size", "bd_confidence_select",
             "bd_block_mask_attn", "bd_status_string", "bd_last_cuda_error_string",
-            "bd_kernel_launches", "bd_confidence_select_noalloc", "bd_confidence_select_active")
+            "bd_kernel_launches", "bd_confidence_select_noalloc", "bd_confidence_select_active",
+            "bd_masked_ce_workspace_size", "bd_masked_ce")
 BD_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 if not os.path.exists(_LIB_PATH):
@@ -71,6 +72,8 @@ _SIGS = {
                                      _P, _P, _P],
     "bd_confidence_select_active": [_I, _I, _I, _I, _P, _P, _P, _P, ctypes.c_float, _I, _P, _P,
                                     _P, _P, _P, ctypes.c_size_t, _P],
+    "bd_masked_ce_workspace_size": [_I, _I, _I, _I, _I, _SZ],
+    "bd_masked_ce": [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -199,6 +202,22 @@ def bd_confidence_select_active(dtype, batch, hidden, vocab, h, h_prev, w_lm, ma
         _ptr(w_lm), _ptr(masked_bits), float(tau), int(sub_block), _ptr(tokens),
         _ptr(unmask_bits), _ptr(pmax_out), _ptr(argmax_out), _ptr(workspace), int(wsb),
         _stream(stream)))
+
+
+def bd_masked_ce_workspace_size(dtype, n_seqs, seq_len, hidden, vocab) -> int:
+    n = ctypes.c_size_t(0)
+    _check("bd_masked_ce_workspace_size", _lib.bd_masked_ce_workspace_size(
+        dtype_code(dtype), int(n_seqs), int(seq_len), int(hidden), int(vocab), ctypes.byref(n)))
+    return int(n.value)
+
+
+def bd_masked_ce(dtype, n_seqs, seq_len, hidden, vocab, h, w_lm, targets, masked_bits, loss_out,
+                 loss_sum, n_scored, workspace, workspace_bytes=None, stream=None):
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check("bd_masked_ce", _lib.bd_masked_ce(
+        dtype_code(dtype), int(n_seqs), int(seq_len), int(hidden), int(vocab), _ptr(h),
+        _ptr(w_lm), _ptr(targets), _ptr(masked_bits), _ptr(loss_out), _ptr(loss_sum),
+        _ptr(n_scored), _ptr(workspace), int(wsb), _stream(stream)))
 
 
 def bd_confidence_select_noalloc(dtype, batch, hidden, vocab, h, h_prev, w_lm, masked_bits, tau,

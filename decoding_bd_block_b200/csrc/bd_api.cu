@@ -208,6 +208,36 @@ int bd_confidence_select_active(int32_t dtype, int32_t batch, int32_t hidden, in
                            tokens, unmask_bits, pmax_out, argmax_out, ws, ws_bytes, stream, 1);
 }
 
+int bd_masked_ce_workspace_size(int32_t dtype, int32_t n_seqs, int32_t seq_len, int32_t hidden,
+                                int32_t vocab, size_t* bytes) {
+  if (!bytes || n_seqs <= 0 || seq_len <= 0 || hidden <= 0 || vocab <= 0) return BD_ERR_INVALID_ARG;
+  if (dtype != BD_F32 && dtype != BD_BF16) return BD_ERR_UNSUPPORTED;
+  if (seq_len % bd::kBlock != 0 || hidden % 8 != 0) return BD_ERR_UNSUPPORTED;
+  if (static_cast<long long>(n_seqs) * seq_len > (1LL << 30)) return BD_ERR_INVALID_ARG;
+  *bytes = bd::plan_masked_ce(dtype, n_seqs, seq_len, hidden, vocab).total;
+  return BD_OK;
+}
+
+int bd_masked_ce(int32_t dtype, int32_t n_seqs, int32_t seq_len, int32_t hidden, int32_t vocab,
+                 const void* h, const void* w, const int32_t* targets,
+                 const uint32_t* masked_bits, float* loss_out, float* loss_sum, int32_t* n_scored,
+                 void* ws, size_t ws_bytes, void* stream) {
+  if (n_seqs <= 0 || seq_len <= 0 || hidden <= 0 || vocab <= 0) return BD_ERR_INVALID_ARG;
+  if (dtype != BD_F32 && dtype != BD_BF16) return BD_ERR_UNSUPPORTED;
+  if (seq_len % bd::kBlock != 0 || hidden % 8 != 0) return BD_ERR_UNSUPPORTED;
+  if (static_cast<long long>(n_seqs) * seq_len > (1LL << 30)) return BD_ERR_INVALID_ARG;
+  if (!h || !w || !targets || !masked_bits || !loss_sum) return BD_ERR_INVALID_ARG;
+  // rows are copied and W rows read in 16-byte vectors; W is read by TMA
+  if ((reinterpret_cast<uintptr_t>(h) | reinterpret_cast<uintptr_t>(w)) % 16 != 0)
+    return BD_ERR_INVALID_ARG;
+  const bd::CePlan p = bd::plan_masked_ce(dtype, n_seqs, seq_len, hidden, vocab);
+  if (!ws || ws_bytes < p.total) return BD_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return BD_ERR_WORKSPACE;
+  return cuda_status(bd::launch_masked_ce(dtype, n_seqs, seq_len, hidden, vocab, p, h, w, targets,
+                                          masked_bits, loss_out, loss_sum, n_scored, ws,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 int bd_block_mask_attn(const bd_attn_shape* sh, const void* q, const void* k, const void* v,
                        void* out, int32_t n_seqs, int32_t L, int32_t block, void* stream) {
   int st = check_shape(sh);

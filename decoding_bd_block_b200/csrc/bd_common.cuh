@@ -168,6 +168,13 @@ __device__ __forceinline__ uint32_t scored_bits(uint32_t bits, int S, int active
   return bits & win;
 }
 
+// Cross-entropy rows of a training batch: word x of the mask bits covers
+// positions 32 (x mod seq_words) .. +31 of one sequence; position 0 of a
+// sequence has no previous hidden row and is not scored.
+__device__ __forceinline__ uint32_t ce_scored_bits(uint32_t bits, int x, int seq_words) {
+  return x % seq_words == 0 ? bits & ~1u : bits;
+}
+
 // "No decision" for sequence s (a bounded wait gave up): nothing is
 // unmasked, p_max is NaN and the token -2.  Lane i of one warp writes position i.
 __device__ __forceinline__ void no_decision_sequence(int s, uint32_t* unmask, float* pmax_out,
@@ -245,9 +252,12 @@ cudaError_t launch_block_attn(const bd_attn_shape& sh, const bd_kv_cache& c, con
 // Tensor-core LM head (select_tc.cu): persistent grid size and launcher.
 // The packed-row count is the popcount of masked[0 .. batch).
 int lmhead_tc_grid();
+// seq_words > 0: the rows are cross-entropy rows (ce_scored_bits of the
+// batch words), S and active unused.
 cudaError_t launch_lmhead_tc(const void* rows, const void* w, const uint32_t* masked, int batch,
                              int S, int active, int H, int V, int rows_alloc, int part_stride,
-                             float* pm, float* ps, int32_t* pa, int32_t* status, cudaStream_t st);
+                             float* pm, float* ps, int32_t* pa, int32_t* status, cudaStream_t st,
+                             int seq_words = 0);
 
 struct SelectPlan {
   bool fused;        // one kernel, rows resident in shared memory (select_fused.cu)
@@ -282,6 +292,25 @@ bool mask_attn_tc_supported(const bd_attn_shape& sh, int L);
 cudaError_t launch_mask_attn_tc(const bd_attn_shape& sh, const void* q, const void* k,
                                 const void* v, void* out, int n_seqs, int L, int block,
                                 int32_t* status, cudaStream_t st);
+
+// CUDA-core LM head (select_simt.cu): partials [row][n_split] of the first
+// count[0] rows; n_split from lmhead_simt_splits.
+cudaError_t launch_lmhead_simt(int dtype, const void* rows, const void* w, const int32_t* count,
+                               int H, int V, int n_split, int rows_alloc, float* pm, float* ps,
+                               int32_t* pa, cudaStream_t st);
+int lmhead_simt_splits(int vocab, int rows_alloc);
+
+// Masked-token cross-entropy (masked_ce.cu).
+struct CePlan {
+  bool tc;
+  int n_split, rows_alloc;
+  size_t off_count, off_rows, off_rowpos, off_tgt, off_pm, off_ps, off_pa, off_loss, total;
+};
+CePlan plan_masked_ce(int dtype, int n_seqs, int seq_len, int hidden, int vocab);
+cudaError_t launch_masked_ce(int dtype, int n_seqs, int seq_len, int hidden, int vocab,
+                             const CePlan& p, const void* h, const void* w, const int32_t* targets,
+                             const uint32_t* masked, float* loss_out, float* loss_sum,
+                             int32_t* n_scored, void* ws, cudaStream_t st);
 
 cudaError_t launch_block_mask_attn(const bd_attn_shape& sh, const void* q, const void* k,
                                    const void* v, void* out, int n_seqs, int L, int block,

@@ -185,6 +185,32 @@ __global__ void __launch_bounds__(1024) merge_select_kernel(
 }
 
 // -------------------------------------------------------------- host side
+cudaError_t launch_lmhead_simt(int dtype, const void* rows, const void* w, const int32_t* count,
+                               int H, int V, int n_split, int rows_alloc, float* pm, float* ps,
+                               int32_t* pa, cudaStream_t st) {
+  if (dtype == BD_BF16)
+    lmhead_simt_kernel<bf16><<<dim3(n_split, rows_alloc / 32), 256, 0, st>>>(
+        static_cast<const bf16*>(rows), static_cast<const bf16*>(w), count, H, V, n_split, pm, ps,
+        pa);
+  else
+    lmhead_simt_kernel<float><<<dim3(n_split, rows_alloc / 32), 256, 0, st>>>(
+        static_cast<const float*>(rows), static_cast<const float*>(w), count, H, V, n_split, pm,
+        ps, pa);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// vocab splits of the CUDA-core LM head: about four CTAs per SM over the
+// (split, 32-row tile) grid
+int lmhead_simt_splits(int vocab, int rows_alloc) {
+  const int vtiles = (vocab + 63) / 64;
+  const int rtiles = rows_alloc / 32;
+  int ns = (4 * 148 + rtiles - 1) / rtiles;
+  if (ns > vtiles) ns = vtiles;
+  if (ns < 1) ns = 1;
+  return ns;
+}
+
 // The tensor-core LM head takes bf16 whenever every row group of <= 256 rows
 // still gets at least one vocab range of its own.
 static bool use_tc(int dtype, int batch) {
@@ -202,12 +228,7 @@ SelectPlan plan_confidence_select(int dtype, int batch, int hidden, int vocab) {
   } else if (p.tc) {
     p.n_split = lmhead_tc_grid();
   } else {
-    const int vtiles = (vocab + 63) / 64;
-    const int rtiles = p.rows_alloc / 32;
-    int ns = (4 * 148 + rtiles - 1) / rtiles;
-    if (ns > vtiles) ns = vtiles;
-    if (ns < 1) ns = 1;
-    p.n_split = ns;
+    p.n_split = lmhead_simt_splits(vocab, p.rows_alloc);
   }
   const size_t es = dtype == BD_BF16 ? 2 : 4;
   size_t off = 0;

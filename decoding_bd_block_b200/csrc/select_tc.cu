@@ -40,6 +40,7 @@ struct SelectTcArgs {
   const uint32_t* masked;  // [batch] masked-position bits: M = total popcount of the scored bits
   int batch;
   int S, active;           // sub-block size; active-only scoring (scored_bits)
+  int seq_words;           // > 0: cross-entropy rows; bit 0 of every seq_words-th word is not scored
   int H, V;
   int rows_alloc;
   int part_stride;  // partials are [row][part]
@@ -72,7 +73,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     int acc = 0;
     for (int x = threadIdx.x; x < a.batch; x += blockDim.x)
-      acc += __popc(scored_bits(a.masked[x], a.S, a.active));
+      acc += __popc(a.seq_words > 0 ? ce_scored_bits(a.masked[x], x, a.seq_words)
+                                    : scored_bits(a.masked[x], a.S, a.active));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) red_a[0][warp] = acc;
@@ -270,14 +272,16 @@ int lmhead_tc_grid() { return lmh::sm_count(); }
 
 cudaError_t launch_lmhead_tc(const void* rows, const void* w, const uint32_t* masked, int batch,
                              int S, int active, int H, int V, int rows_alloc, int part_stride,
-                             float* pm, float* ps, int32_t* pa, int32_t* status, cudaStream_t st) {
+                             float* pm, float* ps, int32_t* pa, int32_t* status, cudaStream_t st,
+                             int seq_words) {
   CUtensorMap tm_w, tm_w16, tm_rows;
   if (!lmh::make_tmap_2d(&tm_w, w, static_cast<uint64_t>(V), static_cast<uint64_t>(H), kVTile) ||
       !lmh::make_tmap_2d(&tm_w16, w, static_cast<uint64_t>(V), static_cast<uint64_t>(H), 16) ||
       !lmh::make_tmap_2d(&tm_rows, rows, static_cast<uint64_t>(rows_alloc), static_cast<uint64_t>(H),
                     16))
     return cudaErrorInvalidValue;
-  SelectTcArgs a{masked, batch, S, active, H, V, rows_alloc, part_stride, pm, ps, pa, status};
+  SelectTcArgs a{masked, batch, S, active, seq_words, H, V, rows_alloc, part_stride, pm, ps, pa,
+                 status};
   cudaFuncSetAttribute(lmhead_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        kSmemBytes + 1024);
   const cudaError_t e = launch_pdl(lmhead_tc_kernel, dim3(lmhead_tc_grid()), dim3(kThreads),

@@ -173,6 +173,33 @@ MASK_ATTN = MaskAttnConfig(
     name="mask_attn_n8x2_L2048", samples=8, views=2, L=2048, block=32,
     n_heads_q=12, n_heads_kv=2, head_dim=128, seed=1005)
 
+@dataclasses.dataclass(frozen=True)
+class CeConfig:
+    """Training masked-token cross-entropy workload: samples x views
+    sequences of L positions; view 0 masks m ~ Bernoulli(mask_p) per
+    position, view 1 the complement."""
+    name: str
+    samples: int
+    views: int
+    L: int
+    hidden: int
+    vocab: int
+    w_std: float = 0.02
+    s_max: float = 30.0
+    mask_p: float = 0.5
+    seed: int = 0
+    dtype: str = "bf16"
+
+    @property
+    def n_seqs(self) -> int:
+        return self.samples * self.views
+
+
+# The training batch of the mask-attention workload (8 samples x 2 views,
+# L = 2048) with the LM head of the 1.5B-shaped decoding workload.
+MASKED_CE = CeConfig(name="masked_ce_n8x2_L2048", samples=8, views=2, L=2048, hidden=1536,
+                     vocab=151936, seed=1006)
+
 STEP_CONFIGS = {c.name: c for c in
                 (TINY_F32, TINY_F32_LITERAL, QWEN15B_STEP, QWEN7B_RAGGED,
                  LONGCTX_ATTN)}
@@ -304,3 +331,45 @@ def make_mask_attn_inputs(cfg: MaskAttnConfig):
         out[name] = t.reshape(S * V, 2 * L, H, d)
     out["m"] = m
     return out
+
+
+def make_ce_inputs(cfg: CeConfig):
+    """h ``[N, L, H]``, W ``[V, H]``, targets ``[N, L]``, masked bits
+    ``[N, L/32]`` for N = samples x views.
+
+    Targets x_0 ~ U{0..V-1} per sample (shared by its views).  Row i-1 of
+    every sequence is a planted peak toward the target of position i,
+    h = s * W[y] / ||W[y]|| + N(0, I) with s ~ U(0, s_max), so the losses
+    range from about log V down to near 0.  View 0 masks position i with
+    probability mask_p, view 1 the complement.
+    """
+    S, V_, L, H, V = cfg.samples, cfg.views, cfg.L, cfg.hidden, cfg.vocab
+    N = S * V_
+    W = normal(_stream(cfg.seed, 60), (V, H), cfg.w_std, cfg.dtype)
+    rng = np.random.Generator(np.random.PCG64(_stream(cfg.seed, 61)))
+    y = rng.integers(0, V, size=(S, L)).astype(np.int32)
+    m = rng.random((S, L)) < cfg.mask_p
+    strength = rng.uniform(0.0, cfg.s_max, size=(N, L)).astype(np.float32)
+    targets = np.repeat(y, V_, axis=0)                       # [N, L]
+    # row i-1 points at the target of position i (the last row at a random token)
+    nxt = np.concatenate([targets[:, 1:], rng.integers(0, V, size=(N, 1)).astype(np.int32)], 1)
+    h = np.empty((N, L, H), dtype=np.uint16 if cfg.dtype == "bf16" else np.float32)
+    chunk = max(1, (1 << 22) // H)
+    flat_t = nxt.reshape(-1)
+    flat_s = strength.reshape(-1)
+    out = h.reshape(N * L, H)
+    for r0 in range(0, N * L, chunk):
+        r1 = min(N * L, r0 + chunk)
+        Wt = as_f32(W[flat_t[r0:r1]], cfg.dtype)
+        nrm = np.sqrt((Wt.astype(np.float64) ** 2).sum(-1, keepdims=True)).astype(np.float32)
+        noise = normal([cfg.seed, 62, r0], (r1 - r0, H), 1.0, "f32")
+        rows = (flat_s[r0:r1, None] * Wt / nrm + noise).astype(np.float32)
+        out[r0:r1] = bf16_bits_from_f32(rows) if cfg.dtype == "bf16" else rows
+    mv = np.empty((N, L), dtype=bool)
+    for smp in range(S):
+        for view in range(V_):
+            mv[smp * V_ + view] = m[smp] if view % 2 == 0 else ~m[smp]
+    bits = np.zeros((N, L // BLOCK), dtype=np.uint32)
+    for k in range(BLOCK):
+        bits |= (mv[:, k::BLOCK].astype(np.uint32) << np.uint32(k))
+    return dict(h=h, W=W, targets=targets, masked_bits=bits, mask=mv)

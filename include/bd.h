@@ -199,6 +199,40 @@ BD_API int bd_confidence_select_active(int32_t dtype, int32_t batch, int32_t hid
                                 int32_t* argmax_out, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* bd_masked_ce -- masked-token cross-entropy of training, logits on chip.
+ *
+ * [N1] key design 2, the L_block equation with the shifted label: in each of
+ * n_seqs training sequences of seq_len positions (the noisy stream x_t),
+ * every position i >= 1 whose token is [MASK] contributes
+ *     -log softmax(W h_{i-1})[x_0^i]  =  max l + log sum exp(l - max) - l_y,
+ * l = W h_{i-1}; position 0 of a sequence has no previous row and is not
+ * scored.  The expectation of the equation is left to the caller.
+ *
+ *   h            device, [n_seqs][seq_len][hidden]: final hidden rows of x_t
+ *   w_lm         device, [vocab][hidden]
+ *   targets      device, [n_seqs][seq_len] int32: the clean tokens x_0
+ *   masked_bits  device, [n_seqs][seq_len / 32] uint32: bit i % 32 of word
+ *                i / 32 set = position i is [MASK] in x_t
+ *   loss_out     device, [n_seqs][seq_len] float or NULL: the loss at every
+ *                scored position, NaN elsewhere
+ *   loss_sum     device, [1] float: the sum over the scored positions (added
+ *                in a fixed order: the same inputs give the same bits)
+ *   n_scored     device, [1] int32 or NULL: the number of scored positions
+ * seq_len % 32 == 0; hidden % 8 == 0; h and w_lm 16-byte aligned.  A target
+ * outside [0, vocab) gives a NaN loss.  Workspace:
+ * bd_masked_ce_workspace_size() bytes, 256-byte aligned.  bf16 with up to
+ * 148 x 256 positions runs the LM head on the tensor cores; if one of its
+ * bounded waits ever gives up, every loss is NaN. */
+BD_API int bd_masked_ce_workspace_size(int32_t dtype, int32_t n_seqs,
+                                int32_t seq_len, int32_t hidden, int32_t vocab,
+                                size_t* bytes);
+BD_API int bd_masked_ce(int32_t dtype, int32_t n_seqs, int32_t seq_len,
+                 int32_t hidden, int32_t vocab, const void* h,
+                 const void* w_lm, const int32_t* targets,
+                 const uint32_t* masked_bits, float* loss_out, float* loss_sum,
+                 int32_t* n_scored, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
 /* bd_confidence_select_noalloc -- bd_confidence_select without a workspace.
  *
  * The method's description has no counterpart to this call: it exists for
