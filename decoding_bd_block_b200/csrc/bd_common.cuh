@@ -302,10 +302,17 @@ int lmhead_simt_splits(int vocab, int rows_alloc);
 
 // Masked-token cross-entropy (masked_ce.cu).
 struct CePlan {
-  bool tc;
+  bool tc;    // LM head on tcgen05 with W as the M operand (few rows)
+  bool rows;  // LM head on tcgen05 with the rows as the M operand (many rows)
   int n_split, rows_alloc;
   size_t off_count, off_rows, off_rowpos, off_tgt, off_pm, off_ps, off_pa, off_loss, total;
 };
+// Rows-as-M LM head of the cross-entropy (ce_lmhead.cu): (max, sum exp)
+// partials [row][R] over R vocab ranges; bf16, rows_alloc a multiple of 256.
+int lmhead_rows_ranges(int vocab);
+cudaError_t launch_lmhead_rows(const void* rows, const void* w, const uint32_t* masked,
+                               int n_words, int seq_words, int H, int V, int rows_alloc, int R,
+                               float* pm, float* ps, int32_t* status, cudaStream_t st);
 CePlan plan_masked_ce(int dtype, int n_seqs, int seq_len, int hidden, int vocab);
 cudaError_t launch_masked_ce(int dtype, int n_seqs, int seq_len, int hidden, int vocab,
                              const CePlan& p, const void* h, const void* w, const int32_t* targets,

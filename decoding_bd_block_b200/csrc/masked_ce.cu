@@ -14,7 +14,8 @@
 //                  the position and its target per packed row; writes NaN
 //                  to the loss of every unscored position;
 //   2. LM head     (max, sum exp) per packed row, vocab-split partials
-//                  (tcgen05 for bf16, CUDA cores for fp32);
+//                  (tcgen05 for bf16: rows as the M operand from 2048 rows
+//                  up, W as the M operand below; CUDA cores for fp32);
 //   3. ce_merge    per row: merge the partials, the target logit as a dot
 //                  product of W[y] and the row, the loss;
 //   4. ce_sum      one CTA adds the losses in row order (a deterministic
@@ -162,6 +163,13 @@ __global__ void __launch_bounds__(1024) ce_sum_kernel(const float* __restrict__ 
   }
 }
 
+// bf16 LM head: rows as the MMA's M operand from 2048 packed rows up (W is
+// then streamed about once); below that W as the M operand, the rows
+// re-read per vocab tile.
+constexpr int kCeRowsMin = 2048;
+bool ce_use_rows(int dtype, int rows_alloc) {
+  return dtype == BD_BF16 && rows_alloc >= kCeRowsMin;
+}
 bool ce_use_tc(int dtype, int rows_alloc) {
   return dtype == BD_BF16 && (rows_alloc + 255) / 256 <= lmhead_tc_grid();
 }
@@ -172,8 +180,10 @@ CePlan plan_masked_ce(int dtype, int n_seqs, int seq_len, int hidden, int vocab)
   CePlan p{};
   const size_t positions = static_cast<size_t>(n_seqs) * seq_len;
   p.rows_alloc = static_cast<int>(align_up(positions, 256));
-  p.tc = ce_use_tc(dtype, p.rows_alloc);
-  p.n_split = p.tc ? lmhead_tc_grid() : lmhead_simt_splits(vocab, p.rows_alloc);
+  p.rows = ce_use_rows(dtype, p.rows_alloc);
+  p.tc = !p.rows && ce_use_tc(dtype, p.rows_alloc);
+  p.n_split = p.rows ? lmhead_rows_ranges(vocab)
+                     : (p.tc ? lmhead_tc_grid() : lmhead_simt_splits(vocab, p.rows_alloc));
   const size_t es = dtype == BD_BF16 ? 2 : 4;
   const size_t ra = static_cast<size_t>(p.rows_alloc);
   size_t off = 0;
@@ -219,7 +229,10 @@ static cudaError_t launch_ce_t(int n_seqs, int seq_len, int hidden, int vocab, c
                              rows, rowpos, tgt, count, loss_out, p.rows_alloc);
   if (e != cudaSuccess) return e;
   count_launches(1);
-  if (p.tc) {
+  if (p.rows) {
+    e = launch_lmhead_rows(rows, w, masked, n_words, seq_words, hidden, vocab, p.rows_alloc,
+                           p.n_split, pm, ps, count + 1, st);
+  } else if (p.tc) {
     e = launch_lmhead_tc(rows, w, masked, n_words, kBlock, 0, hidden, vocab, p.rows_alloc,
                          p.n_split, pm, ps, pa, count + 1, st, seq_words);
   } else {

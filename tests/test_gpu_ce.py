@@ -52,6 +52,11 @@ SMALL = [
                         vocab=1001, seed=203),
     dataclasses.replace(W.MASKED_CE, name="bf16_all_masked", samples=1, views=1, L=64, hidden=256,
                         vocab=777, mask_p=1.0, seed=204),
+    # >= 2048 packed rows: the rows-as-M LM head; ragged K (264 = 4 x 64 + 8),
+    # ragged last W tile (20001 = 78 x 256 + 33), 9 vocab ranges, a partial
+    # last row pair
+    dataclasses.replace(W.MASKED_CE, name="bf16_rows_s2x2_L1024", samples=2, L=1024, hidden=264,
+                        vocab=20001, seed=206),
 ]
 
 
