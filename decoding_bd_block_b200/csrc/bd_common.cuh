@@ -308,7 +308,7 @@ struct CePlan {
   size_t off_count, off_rows, off_rowpos, off_tgt, off_pm, off_ps, off_pa, off_loss, total;
 };
 // Rows-as-M LM head of the cross-entropy (ce_lmhead.cu): (max, sum exp)
-// partials [row][R] over R vocab ranges; bf16, rows_alloc a multiple of 256.
+// partials [row][2 R] over R vocab ranges; bf16, rows_alloc a multiple of 256.
 int lmhead_rows_ranges(int vocab);
 cudaError_t launch_lmhead_rows(const void* rows, const void* w, const uint32_t* masked,
                                int n_words, int seq_words, int H, int V, int rows_alloc, int R,

@@ -15,18 +15,20 @@
 //     vocab ranges: W comes from HBM about once, the rows (they fit in L2)
 //     from L2.
 //   * warp 0 streams the stages by TMA (3 stages), warp 1 issues tcgen05.mma
-//     into two 256-column TMEM accumulators (one per row tile), warps 2-9
-//     each drain 32 rows x 256 columns after a W tile; a thread owns one row,
+//     into two 256-column TMEM accumulators (one per row tile), warps 2-17
+//     each drain 32 rows x 128 columns after a W tile; a thread owns one row,
 //     so the fold into its running (max, sum exp) needs no shuffles.  The
 //     accumulators are not double-buffered (2 x 256 columns fill TMEM): the
-//     MMA waits for each drain.
-//   * per unit, each row gets one (max, sum exp) partial: [row][R].
+//     MMA waits for each drain, so the drain is spread over 16 warps with
+//     the next TMEM load in flight during each fold.
+//   * per unit, each row gets two (max, sum exp) partials, one per column
+//     half: [row][2 R].
 #include "lmhead_common.cuh"
 
 namespace bd {
 namespace {
 
-constexpr int kThreads = 320;                 // 10 warps
+constexpr int kThreads = 576;                 // 18 warps
 constexpr int kRowTile = 128;                 // MMA M
 constexpr int kWTile = 256;                   // MMA N: vocab rows per W tile
 constexpr int kK = 64;                        // hidden elements per stage
@@ -41,11 +43,38 @@ struct RowsArgs {
   const uint32_t* masked;  // mask words of the batch (ce_scored_bits)
   int n_words, seq_words;
   int H, V;
-  int R;                   // vocab ranges (partials per row)
-  float* pm;               // [row][R]
+  int R;                   // vocab ranges (2 R partials per row)
+  float* pm;               // [row][2 R]
   float* ps;
   int32_t* status;
 };
+
+// Folds 32 logits (the first n valid; kFull: all 32) into a running
+// (max, sum exp).
+template <bool kFull>
+__device__ __forceinline__ void fold32(const uint32_t (&r)[32], int n, float& run_m,
+                                       float& run_s) {
+  float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float x = (kFull || i < n) ? __uint_as_float(r[i]) : -INFINITY;
+    mk[i & 3] = fmaxf(mk[i & 3], x);
+  }
+  const float m_new = fmaxf(run_m, fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])));
+  if (m_new == -INFINITY) return;
+  const float mls = m_new * kLog2e;
+  float sk[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (kFull || i < n) {
+      const float y = fmaf(__uint_as_float(r[i]), kLog2e, -mls);
+      // one exponential in four on the FMA pipe, the rest on MUFU
+      sk[i & 3] += (i & 3) == 3 ? poly_exp2(y) : fast_exp2(y);
+    }
+  }
+  run_s = run_s * fast_exp2((run_m - m_new) * kLog2e) + ((sk[0] + sk[1]) + (sk[2] + sk[3]));
+  run_m = m_new;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     lmhead_rows_kernel(const __grid_constant__ CUtensorMap tm_rows,
@@ -73,7 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&empty_bar[s], 1);
     }
     tc::mbar_init(&tfull_bar, 1);
-    tc::mbar_init(&tempty_bar, 8);
+    tc::mbar_init(&tempty_bar, 16);
     tc::mbar_init(&done_bar, 1);
     tc::fence_barrier_init();
     tc::fence_proxy_async();
@@ -172,10 +201,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------- epilogue
-    // warps 2..9: row tile tt, TMEM lane quarter q (= warp % 4, the lanes
-    // this warp may access); one row per thread
-    const int tt = (warp - 2) / 4, q = warp & 3;
-    const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + tt * kWTile;
+    // warps 2..17 (e = warp - 2): row tile tt, column half hf of the W tile,
+    // TMEM lane quarter q (= warp % 4, the lanes this warp may access); one
+    // row per thread, four 32-column chunks per W tile, the load of the next
+    // chunk in flight while this one is folded
+    const int e = warp - 2, tt = (e >> 2) & 1, hf = e >> 3, q = warp & 3;
+    const uint32_t tbase =
+        tmem + (static_cast<uint32_t>(q * 32) << 16) + tt * kWTile + hf * (kWTile / 2);
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -187,43 +219,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int wt = wt0; wt < wt1; ++wt, ++it) {
         if (!tc::mbar_wait_warp(&tfull_bar, it & 1, a.status)) { ok = false; break; }
         tc::tc_fence_after();
-        const int vend = min(kWTile, a.V - wt * kWTile);  // valid columns of this W tile
-#pragma unroll 1
-        for (int c = 0; c * 32 < vend; ++c) {  // warp-uniform trip count
-          uint32_t r[32];
-          tc::tmem_ld_32x32b_x32(tbase + c * 32, r);
-          tc::tmem_ld_wait();
-          const bool full = (c + 1) * 32 <= vend;
-          float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        // valid columns of this warp's half of the W tile (warp-uniform)
+        const int lim = min(kWTile, a.V - wt * kWTile) - hf * (kWTile / 2);
+        const int nc = lim <= 0 ? 0 : min(4, (lim + 31) / 32);
+        uint32_t rb[2][32];
+        if (nc > 0) tc::tmem_ld_32x32b_x32(tbase, rb[0]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float x = (full || c * 32 + i < vend) ? __uint_as_float(r[i]) : -INFINITY;
-            mk[i & 3] = fmaxf(mk[i & 3], x);
+        for (int c = 0; c < 4; ++c) {
+          if (c < nc) {
+            tc::tmem_ld_wait(rb[c & 1]);
+            if (c + 1 < nc) tc::tmem_ld_32x32b_x32(tbase + (c + 1) * 32, rb[(c + 1) & 1]);
+            if (lim >= (c + 1) * 32)
+              fold32<true>(rb[c & 1], 32, run_m, run_s);
+            else
+              fold32<false>(rb[c & 1], lim - c * 32, run_m, run_s);
           }
-          const float m_new = fmaxf(run_m, fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])));
-          if (m_new != -INFINITY) {
-            const float mls = m_new * kLog2e;
-            float sk[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float x = (full || c * 32 + i < vend) ? __uint_as_float(r[i]) : -INFINITY;
-              const float y = fmaf(x, kLog2e, -mls);
-              // 3 of 8 exponentials on the FMA pipe, the rest on MUFU
-              sk[i & 3] += (i & 7) < 3 ? poly_exp2(y) : fast_exp2(y);
-            }
-            run_s = run_s * fast_exp2((run_m - m_new) * kLog2e) +
-                    ((sk[0] + sk[1]) + (sk[2] + sk[3]));
-            run_m = m_new;
-          }
-          __syncwarp();
         }
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&tempty_bar);
       }
       if (ok && row < M) {
-        a.pm[static_cast<size_t>(row) * a.R + v] = run_m;
-        a.ps[static_cast<size_t>(row) * a.R + v] = run_s;
+        a.pm[static_cast<size_t>(row) * 2 * a.R + 2 * v + hf] = run_m;
+        a.ps[static_cast<size_t>(row) * 2 * a.R + 2 * v + hf] = run_s;
       }
     }
   }
@@ -235,6 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+// Partials per row = 2 x the vocab ranges.
 int lmhead_rows_ranges(int vocab) {
   // about 8 W tiles per unit, at most 64 partials per row
   const int n_wt = (vocab + kWTile - 1) / kWTile;

@@ -182,7 +182,7 @@ CePlan plan_masked_ce(int dtype, int n_seqs, int seq_len, int hidden, int vocab)
   p.rows_alloc = static_cast<int>(align_up(positions, 256));
   p.rows = ce_use_rows(dtype, p.rows_alloc);
   p.tc = !p.rows && ce_use_tc(dtype, p.rows_alloc);
-  p.n_split = p.rows ? lmhead_rows_ranges(vocab)
+  p.n_split = p.rows ? 2 * lmhead_rows_ranges(vocab)
                      : (p.tc ? lmhead_tc_grid() : lmhead_simt_splits(vocab, p.rows_alloc));
   const size_t es = dtype == BD_BF16 ? 2 : 4;
   const size_t ra = static_cast<size_t>(p.rows_alloc);
@@ -231,7 +231,7 @@ static cudaError_t launch_ce_t(int n_seqs, int seq_len, int hidden, int vocab, c
   count_launches(1);
   if (p.rows) {
     e = launch_lmhead_rows(rows, w, masked, n_words, seq_words, hidden, vocab, p.rows_alloc,
-                           p.n_split, pm, ps, count + 1, st);
+                           p.n_split / 2, pm, ps, count + 1, st);
   } else if (p.tc) {
     e = launch_lmhead_tc(rows, w, masked, n_words, kBlock, 0, hidden, vocab, p.rows_alloc,
                          p.n_split, pm, ps, pa, count + 1, st, seq_words);
