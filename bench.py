@@ -169,6 +169,14 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+def gpu_uuid(dev):
+    try:
+        import torch
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -515,8 +523,10 @@ def run_mask_attn(args, cfg, dist: Dist):
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     launches0 = bd.bd_kernel_launches()
+    sampler = ClockSampler(gpu_uuid(dev))
     dist.barrier()
     torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
     for i in range(K):
         flush.zero_()
         ev[i][0].record(stream)
@@ -524,6 +534,7 @@ def run_mask_attn(args, cfg, dist: Dist):
         ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     dist.barrier()
+    clocks = sampler.stop(t_wall0, time.time())
     launches = bd.bd_kernel_launches() - launches0
     ms, rows_per_s = replica_throughput(dist, float(cfg.n_seqs * 2 * cfg.L * cfg.n_heads_q),
                                         float(np.mean([e[0].elapsed_time(e[1]) for e in ev])), dev)
@@ -546,6 +557,7 @@ def run_mask_attn(args, cfg, dist: Dist):
                      "traffic": recorded_traffic("mask_attn"),
                      "algorithmic_flop_per_launch": flop, "peak_source": peak_kind},
         "gpu_launches": int(launches),
+        "clocks": clocks,
     }
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
@@ -583,8 +595,10 @@ def run_masked_ce(args, cfg, dist: Dist):
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     launches0 = bd.bd_kernel_launches()
+    sampler = ClockSampler(gpu_uuid(dev))
     dist.barrier()
     torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
     for i in range(K):
         flush.zero_()
         ev[i][0].record(stream)
@@ -592,12 +606,14 @@ def run_masked_ce(args, cfg, dist: Dist):
         ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     dist.barrier()
+    clocks = sampler.stop(t_wall0, time.time())
     launches = bd.bd_kernel_launches() - launches0
     ms, value = replica_throughput(dist, float(count),
                                    float(np.mean([e[0].elapsed_time(e[1]) for e in ev])), dev)
     flop = 2.0 * count * cfg.vocab * cfg.hidden
     peaks, peak_kind = measured_peaks()
     peak = float(peaks.get("bf16_tflops", 1590.0))
+    peak_sus = peaks.get("bf16_tflops_sustained")
     ach = flop / (ms / 1e3) / 1e12
     line = {
         "metric": "masked positions' cross-entropy computed/s (training batch)",
@@ -611,8 +627,10 @@ def run_masked_ce(args, cfg, dist: Dist):
         "roofline": {"kernel": "bd_masked_ce (LM head on tcgen05; whole call timed)",
                      "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                      "frac": ach / peak, "traffic": recorded_traffic("masked_ce"),
-                     "algorithmic_flop_per_launch": flop, "peak_source": peak_kind},
+                     "algorithmic_flop_per_launch": flop, "peak_source": peak_kind,
+                     "frac_of_sustained_peak": (ach / float(peak_sus)) if peak_sus else None},
         "gpu_launches": int(launches),
+        "clocks": clocks,
     }
     if dist.rank == 0:
         print(json.dumps(line), flush=True)

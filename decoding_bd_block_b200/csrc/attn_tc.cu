@@ -7,8 +7,11 @@
 // CTA = (split-KV chunk, KV head g, sequence s).  Its query rows are the
 // G = Hq/Hkv heads of group g times the block's 32 positions (row r = head
 // (r / 32) of the group, position r % 32), one or two 128-row tiles Q_t,
-// loaded once by TMA into shared memory.  The chunk's pages stream through
-// two 128-key K/V stages (four pages per stage, TMA, 128-byte swizzle).
+// loaded once by TMA into shared memory.  The chunk's pages stream in
+// 128-key steps (four pages, TMA, 128-byte swizzle) through a ring of four
+// 32 KB slots holding K_0, V_0, K_1, V_1, K_2, ... in turn: K_j's slot is
+// released as soon as S(j) = Q K_j^T has been computed, V_j's after P V_j,
+// so the loads of step j+2 start about two steps before they are needed.
 //
 // Tensor memory (512 columns): S_t at 128 t (fp32; P_t is written over its
 // first 64 columns as packed bf16), O_t at 256 + 128 t (fp32).
@@ -41,8 +44,9 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kThreads = 384;               // 12 warps
-constexpr int kKeys = 128;                   // keys per stage (four pages)
-constexpr int kStages = 2;
+constexpr int kKeys = 128;                   // keys per step (four pages)
+constexpr int kSlots = 4;                    // ring slots of one K or V step each
+constexpr int kPreSteps = kSlots / 2;        // steps whose slots are free at the start
 constexpr int kQTileBytes = 128 * kD * 2;    // 32 KB
 constexpr int kKVBytes = kKeys * kD * 2;     // 32 KB each for K and V
 constexpr int kMaxChunkPages = 1024;
@@ -51,7 +55,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr int kOffQ = 0;
 constexpr int kOffKV = 2 * kQTileBytes;
-constexpr int kSmemBytes = kOffKV + kStages * 2 * kKVBytes + 1024;  // + alignment slack
+constexpr int kSmemBytes = kOffKV + kSlots * kKVBytes + 1024;  // + alignment slack
 
 struct AttnTcArgs {
   const int32_t* page_table;
@@ -76,7 +80,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   __shared__ uint64_t q_full;
-  __shared__ uint64_t kv_full[kStages], kv_empty[kStages];
+  __shared__ uint64_t kv_full[kSlots], kv_empty[kSlots];
   __shared__ uint64_t s_full[2], p_full[2], pv_done[2];
   __shared__ uint32_t tmem_slot;
   __shared__ int pages[kMaxChunkPages];
@@ -106,7 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (threadIdx.x == 0) {
     tc::mbar_init(&q_full, 1);
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kSlots; ++i) {
       tc::mbar_init(&kv_full[i], 1);
       tc::mbar_init(&kv_empty[i], 1);
     }
@@ -156,43 +160,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     };
     const bool has_blk = p1 == total;  // the chunk ends with the current block's page
-    const int pg = (lane >> 2) & 3, kv = (lane >> 1) & 1, dh = lane & 1;
-    int st = 0;
-    uint32_t ph = 0;
-    for (int j = 0; j < n_tiles; ++j) {
-      if (!dep && (j >= kStages || (has_blk && j == n_tiles - 1))) wait_prep_load_q();
-      if (!tc::mbar_wait_warp(&kv_empty[st], ph ^ 1, a.status)) break;
-      if (lane == 0) tc::mbar_arrive_expect_tx(&kv_full[st], 2 * kKVBytes);
-      __syncwarp();
-      if (lane < 16) {
-        const int i = 4 * j + pg;
-        const CUtensorMap* m = &tm_kv;
-        int row;
-        if (i >= n_pg || pages[i] == -2) {  // padding page: rows past the end read as zeros
-          row = a.kv_rows_total;
-        } else if (pages[i] == -1) {
-          m = &tm_blk;
-          row = ((s * 2 + kv) * a.Hkv + g) * kBlock;
-        } else {
-          row = ((pages[i] * 2 + kv) * a.Hkv + g) * kBlock;
+    const int pg = (lane >> 1) & 3, dh = lane & 1;
+    bool ok = true;
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      if (!dep && (j >= kPreSteps || (has_blk && j == n_tiles - 1))) wait_prep_load_q();
+      for (int kv = 0; kv < 2; ++kv) {  // K_j, then V_j: ring buffer b = 2 j + kv
+        const int b = 2 * j + kv, sl = b % kSlots;
+        if (!tc::mbar_wait_warp(&kv_empty[sl], ((b / kSlots) & 1) ^ 1, a.status)) {
+          ok = false;
+          break;
         }
-        tc::tma_load_2d(smem + kOffKV + st * 2 * kKVBytes + kv * kKVBytes + dh * (kKVBytes / 2) +
-                            pg * 4096,
-                        m, &kv_full[st], dh * 64, row, pol_kv);
+        if (lane == 0) tc::mbar_arrive_expect_tx(&kv_full[sl], kKVBytes);
+        __syncwarp();
+        if (lane < 8) {  // the step's 8 boxes: 4 pages x 2 halves of d
+          const int i = 4 * j + pg;
+          const CUtensorMap* m = &tm_kv;
+          int row;
+          if (i >= n_pg || pages[i] == -2) {  // padding page: rows past the end read as zeros
+            row = a.kv_rows_total;
+          } else if (pages[i] == -1) {
+            m = &tm_blk;
+            row = ((s * 2 + kv) * a.Hkv + g) * kBlock;
+          } else {
+            row = ((pages[i] * 2 + kv) * a.Hkv + g) * kBlock;
+          }
+          tc::tma_load_2d(smem + kOffKV + sl * kKVBytes + dh * (kKVBytes / 2) + pg * 4096, m,
+                          &kv_full[sl], dh * 64, row, pol_kv);
+        }
+        __syncwarp();
       }
-      if (++st == kStages) { st = 0; ph ^= 1; }
     }
-    // Fewer tiles than stages, none holding the current block (the loop
-    // cannot stop early before `dep`: the first kStages stages are free).
+    // Fewer steps than kPreSteps, none holding the current block (the loop
+    // cannot stop early before `dep`: the first kPreSteps steps' slots are
+    // free).
     if (!dep) wait_prep_load_q();
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_qk = tc::idesc_bf16_f32(128, kKeys);
       const uint32_t id_pv = tc::idesc_bf16_f32_bmn(128, kD);
-      auto issue_qk = [&](int t, int st) {  // S_t = Q_t K^T, K = d: 8 steps of 16
+      auto slot_addr = [&](int b) { return sbase + kOffKV + (b % kSlots) * kKVBytes; };
+      auto full = [&](int b) { return tc::mbar_wait(&kv_full[b % kSlots], (b / kSlots) & 1, a.status); };
+      auto issue_qk = [&](int t, int j) {  // S_t = Q_t K_j^T, K = d: 8 steps of 16
         const uint32_t qaddr = sbase + kOffQ + t * kQTileBytes;
-        const uint32_t kaddr = sbase + kOffKV + st * 2 * kKVBytes;
+        const uint32_t kaddr = slot_addr(2 * j);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (kk & 3) * 32;
@@ -203,18 +214,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::mma_commit(&s_full[t]);
       };
-      bool ok = tc::mbar_wait(&q_full, 0, a.status) && tc::mbar_wait(&kv_full[0], 0, a.status);
+      bool ok = tc::mbar_wait(&q_full, 0, a.status) && full(0);
       tc::tc_fence_after();
       for (int t = 0; t < nq && ok; ++t) issue_qk(t, 0);
-      int st = 0;
-      uint32_t ph = 0;
+      if (ok) tc::mma_commit(&kv_empty[0]);  // K_0 has been read once its products are done
       for (int j = 0; j < n_tiles && ok; ++j) {
-        const int st1 = st + 1 == kStages ? 0 : st + 1;
-        const uint32_t ph1 = st + 1 == kStages ? ph ^ 1 : ph;
         const bool more = j + 1 < n_tiles;
-        const uint32_t vaddr = sbase + kOffKV + st * 2 * kKVBytes + kKVBytes;
+        const uint32_t vaddr = slot_addr(2 * j + 1);
         for (int t = 0; t < nq && ok; ++t) {
           if (!tc::mbar_wait(&p_full[t], j & 1, a.status)) { ok = false; break; }
+          if (t == 0 && !full(2 * j + 1)) { ok = false; break; }
           tc::tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk)  // O_t += P_t V_j, K = keys: 8 steps of 16
@@ -222,15 +231,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc::sdesc_mnmajor_sw128(vaddr + kk * 16 * 128, kKVBytes / 2), id_pv,
                             (j | kk) != 0);
           tc::mma_commit(&pv_done[t]);
+          if (t == nq - 1) tc::mma_commit(&kv_empty[(2 * j + 1) % kSlots]);  // V_j read
           if (more) {
-            if (t == 0 && !tc::mbar_wait(&kv_full[st1], ph1, a.status)) { ok = false; break; }
+            if (t == 0 && !full(2 * j + 2)) { ok = false; break; }
             tc::tc_fence_after();
-            issue_qk(t, st1);
+            issue_qk(t, j + 1);
           }
         }
-        tc::mma_commit(&kv_empty[st]);
-        st = st1;
-        ph = ph1;
+        if (ok && more) tc::mma_commit(&kv_empty[(2 * j + 2) % kSlots]);  // K_{j+1} read
       }
     }
   } else if (warp >= 4 && (warp - 4) / 4 < nq) {
