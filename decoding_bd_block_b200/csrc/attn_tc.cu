@@ -51,6 +51,10 @@ constexpr int kQTileBytes = 128 * kD * 2;    // 32 KB
 constexpr int kKVBytes = kKeys * kD * 2;     // 32 KB each for K and V
 constexpr int kMaxChunkPages = 1024;
 constexpr float kRescaleThreshold = 8.f;     // log2 units
+// pairs of scores whose exponentials are evaluated on the FMA pipe: one in
+// four (a third or a half measured slower: the polynomial's issue cost then
+// outweighs the MUFU time it saves)
+__device__ __forceinline__ constexpr bool kPolyPair(int k) { return (k & 3) == 3; }
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr int kOffQ = 0;
@@ -278,19 +282,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
         m = m_new;
       }
-      const float neg_m = -m;
-      float rk[4] = {0.f, 0.f, 0.f, 0.f};
+      const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(-m, -m);
+      float2 rk[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int k = 0; k < 64; ++k) {  // packs in place: sr[k] <- (p_2k, p_2k+1)
-        // a quarter of the exponentials on the FMA pipe, the rest on MUFU
-        const float x0 = fmaf(__uint_as_float(sr[2 * k]), scale, neg_m);
-        const float x1 = fmaf(__uint_as_float(sr[2 * k + 1]), scale, neg_m);
-        const float e0 = (k & 3) == 3 ? poly_exp2(x0) : fast_exp2(x0);
-        const float e1 = (k & 3) == 3 ? poly_exp2(x1) : fast_exp2(x1);
-        rk[k & 3] += e0 + e1;
-        sr[k] = tc::pack_bf16x2(e0, e1);
+        // paired fp32 arithmetic; a quarter of the pairs' exponentials on the
+        // FMA pipe, the rest on MUFU (the MUFU unit bounds this loop)
+        const float2 x = ffma2(make_float2(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])),
+                               sc2, nm2);
+        const float2 e = kPolyPair(k) ? poly_exp2x2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+        rk[k & 1] = fadd2(rk[k & 1], e);
+        sr[k] = tc::pack_bf16x2(e.x, e.y);
       }
-      l = l * alpha + ((rk[0] + rk[1]) + (rk[2] + rk[3]));
+      l = l * alpha + ((rk[0].x + rk[0].y) + (rk[1].x + rk[1].y));
       // TMEM accesses are warp-collective, so the warp rescales together when
       // any of its rows needs it, the other rows with a factor of 1.
       const bool need = rescale && j > 0;

@@ -53,6 +53,44 @@ __device__ __forceinline__ float poly_exp2(float x) {
   return __int_as_float(__float_as_int(p) + j * (1 << 23));
 }
 
+// Paired fp32 arithmetic (two lanes of a 64-bit register pair per
+// instruction, sm_100): d = a * b + c and d = a + b, each lane rounded as the
+// scalar instruction would be.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+// poly_exp2 on a pair, the polynomial in paired arithmetic.
+__device__ __forceinline__ float2 poly_exp2x2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = fadd2(x, make_float2(12582912.f, 12582912.f));
+  const int jx = __float_as_int(t.x) - 0x4B400000, jy = __float_as_int(t.y) - 0x4B400000;
+  const float2 u = fadd2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = ffma2(u, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(make_float2(0.009570101434f, 0.009570101434f), f,
+                   make_float2(0.05591786028f, 0.05591786028f));
+  p = ffma2(p, f, make_float2(0.2402474484f, 0.2402474484f));
+  p = ffma2(p, f, make_float2(0.6931218147f, 0.6931218147f));
+  p = ffma2(p, f, make_float2(0.9999992614f, 0.9999992614f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + jx * (1 << 23)),
+                     __int_as_float(__float_as_int(p.y) + jy * (1 << 23)));
+}
+
 // ------------------------------------------- programmatic dependent launch
 // A kernel launched with launch_pdl() may start while the previous kernel of
 // the stream is still running: it must call griddep_wait() before it reads

@@ -247,20 +247,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = m_new;
       }
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
-      float rk[4] = {0.f, 0.f, 0.f, 0.f};
+      const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(neg_m, neg_m);
+      float2 rk[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        const float x0 = fmaf(__uint_as_float(sr[2 * k]), scale, neg_m);
-        const float x1 = fmaf(__uint_as_float(sr[2 * k + 1]), scale, neg_m);
-        const float e0 = (k & 3) == 3 ? poly_exp2(x0) : fast_exp2(x0);
-        const float e1 = (k & 3) == 3 ? poly_exp2(x1) : fast_exp2(x1);
-        // poly_exp2 floors at 2^-126 for masked (-inf) scores: exact zeros here
-        const float z0 = (__uint_as_float(sr[2 * k]) == -INFINITY) ? 0.f : e0;
-        const float z1 = (__uint_as_float(sr[2 * k + 1]) == -INFINITY) ? 0.f : e1;
-        rk[k & 3] += z0 + z1;
-        sr[k] = tc::pack_bf16x2(z0, z1);
+      for (int k = 0; k < 64; ++k) {  // packs in place: sr[k] <- (p_2k, p_2k+1)
+        // paired fp32 arithmetic; a quarter of the pairs' exponentials on the
+        // FMA pipe, the rest on MUFU (which gives exact zeros for masked,
+        // -inf, scores; poly_exp2x2 floors at 2^-126, so those are zeroed)
+        const float s0 = __uint_as_float(sr[2 * k]), s1 = __uint_as_float(sr[2 * k + 1]);
+        const float2 x = ffma2(make_float2(s0, s1), sc2, nm2);
+        float2 e;
+        if ((k & 3) == 3) {
+          e = poly_exp2x2(x);
+          e.x = s0 == -INFINITY ? 0.f : e.x;
+          e.y = s1 == -INFINITY ? 0.f : e.y;
+        } else {
+          e = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+        }
+        rk[k & 1] = fadd2(rk[k & 1], e);
+        sr[k] = tc::pack_bf16x2(e.x, e.y);
       }
-      l = l * alpha + ((rk[0] + rk[1]) + (rk[2] + rk[3]));
+      l = l * alpha + ((rk[0].x + rk[0].y) + (rk[1].x + rk[1].y));
       const bool need = rescale && j > 0;
       if (__any_sync(0xffffffffu, need)) {
         const float f = need ? alpha : 1.f;
