@@ -426,7 +426,10 @@ def run_ours(args, cfg, tau, S, dist: Dist):
                           graphs["step"] if graphs else None)
 
     metric, unit = "masked positions scored/s per denoise step", "masked positions scored/s"
-    if step.active_only:
+    if not step.sel:  # attention-only workload: units are (query head, block position) rows
+        metric = "query rows attended/s per denoise step (block attention only)"
+        unit = "query rows/s"
+    elif step.active_only:
         metric = "candidate positions scored/s per denoise step (active sub-block only)"
         unit = "candidate positions scored/s"
     line = {
