@@ -14,6 +14,18 @@ The embedding and projections are torch glue; attention (with RoPE),
 unmask and cache commit are the library's kernels through the C ABI.  A
 finished block is run once more with its final tokens to produce the K/V it
 commits and the last hidden row the next block's position 0 reads.
+
+With ``dual_cache`` the loop keeps the sub-block DualCache of the current
+block (same pages, key design 3; "2.5x inference speedup" article,
+"Acceleration engine" item 1; approximate by the notes' own account): at the
+first step of each active sub-block the whole block is run and its K, V and
+hidden rows are cached; at the following steps of that sub-block only the
+active sub-block's rows are fresh, the attention reading the cached K/V of
+the other rows and the unmask rule the cached hidden rows outside the active
+sub-block.  Only the unmask rule's candidates are scored then
+(``bd_confidence_select_active``).  In this one-layer model the saving the
+cache brings to a deep model (projections and MLPs of the inactive rows) is
+not there to measure; the loop shows the policy and its decisions.
 """
 from __future__ import annotations
 
@@ -67,12 +79,14 @@ def mask_bits(tokens: torch.Tensor) -> torch.Tensor:
 
 
 def decode(model: TinyModel, prompt: np.ndarray, n_blocks: int, tau: float, sub_block: int,
-           device="cuda") -> dict:
-    """Decode n_blocks blocks after a prompt of whole blocks.
+           device="cuda", dual_cache: bool = False) -> dict:
+    """Decode n_blocks blocks after a prompt of whole blocks, exactly or with
+    the sub-block DualCache.
 
     Returns dict(tokens [B, P + 32 n_blocks], steps [n_blocks, B]: denoising
     steps each sequence needed per block, unmasked [n_blocks][step] list of
-    [B] unmask bit words).
+    [B] unmask bit words, refreshes: DualCache refresh steps summed over the
+    sequences).
     """
     cfg = model.cfg
     B, P = prompt.shape
@@ -87,17 +101,24 @@ def decode(model: TinyModel, prompt: np.ndarray, n_blocks: int, tau: float, sub_
                          dtype=torch.uint8, device=device)
     unmask = torch.zeros(B, dtype=torch.int32, device=device)
 
-    def forward(tokens: torch.Tensor):
-        """Hidden rows and pre-RoPE k, v of one block over the current cache."""
+    def project(tokens: torch.Tensor):
         x = w["E"][torch.where(tokens == MASK_TOKEN, torch.full_like(tokens, V), tokens).long()]
         q = (x @ w["Wq"]).view(B, BLOCK, Hq, d).contiguous()
         k = (x @ w["Wk"]).view(B, BLOCK, Hkv, d).contiguous()
         v = (x @ w["Wv"]).view(B, BLOCK, Hkv, d).contiguous()
+        return x, q, k, v
+
+    def attend(x, q, k, v):
+        """Hidden rows of one block over the current cache, given its pre-RoPE k, v."""
         ws = torch.empty(max(bd.bd_block_attn_workspace_size(cache), 256), dtype=torch.uint8,
                          device=device)
-        bd.bd_block_attn(cache, q, k, v, out_blk, ws)
-        h = x + out_blk.view(B, BLOCK, Hq * d) @ w["Wo"]
-        return h.contiguous(), k, v
+        bd.bd_block_attn(cache, q, k.contiguous(), v.contiguous(), out_blk, ws)
+        return (x + out_blk.view(B, BLOCK, Hq * d) @ w["Wo"]).contiguous()
+
+    def forward(tokens: torch.Tensor):
+        """Hidden rows and pre-RoPE k, v of one block over the current cache."""
+        x, q, k, v = project(tokens)
+        return attend(x, q, k, v), k, v
 
     tokens_all = [torch.from_numpy(np.ascontiguousarray(prompt, np.int32)).to(device)]
     h_prev = torch.zeros((B, H), dtype=torch.float32, device=device)
@@ -107,25 +128,49 @@ def decode(model: TinyModel, prompt: np.ndarray, n_blocks: int, tau: float, sub_
         h_prev = h[:, BLOCK - 1].contiguous()
     steps = np.zeros((n_blocks, B), dtype=np.int64)
     unmasked = []
+    refreshes = 0
+    sub_of = torch.arange(BLOCK, device=device) // sub_block
     for b in range(n_blocks):
         tok = torch.full((B, BLOCK), MASK_TOKEN, dtype=torch.int32, device=device)
         log = []
+        cached_sub = torch.full((B,), -1, dtype=torch.long, device=device)
+        Kc = torch.zeros((B, BLOCK, Hkv, d), dtype=torch.float32, device=device)
+        Vc = torch.zeros_like(Kc)
+        Hc = torch.zeros((B, BLOCK, H), dtype=torch.float32, device=device)
         for _ in range(BLOCK + 1):  # at least one token per sequence and step: <= 32 steps
             bits = mask_bits(tok)
             if not bool((tok == MASK_TOKEN).any()):
                 break
             still = (tok == MASK_TOKEN).any(dim=1).cpu().numpy()
             steps[b] += still
-            h, _, _ = forward(tok)
-            bd.bd_confidence_select("f32", B, H, V, h, h_prev, w["W"], bits, tau, sub_block, tok,
-                                    unmask, None, None, sel_ws)
+            if dual_cache:
+                x, q, k, v = project(tok)
+                # active sub-block: the one holding the first masked position
+                a = (tok == MASK_TOKEN).to(torch.int32).argmax(dim=1).long() // sub_block
+                rows = sub_of[None, :] == a[:, None]                      # [B, 32]
+                refresh = cached_sub != a
+                refreshes += int(refresh[torch.from_numpy(still).to(device)].sum())
+                Kc = torch.where(refresh[:, None, None, None], k, Kc)
+                Vc = torch.where(refresh[:, None, None, None], v, Vc)
+                cached_sub = torch.where(refresh, a, cached_sub)
+                h_new = attend(x, q, torch.where(rows[:, :, None, None], k, Kc),
+                               torch.where(rows[:, :, None, None], v, Vc))
+                Hc = torch.where(refresh[:, None, None], h_new, Hc)
+                h = torch.where(rows[:, :, None], h_new, Hc).contiguous()
+                bd.bd_confidence_select_active("f32", B, H, V, h, h_prev, w["W"], bits, tau,
+                                               sub_block, tok, unmask, None, None, sel_ws)
+            else:
+                h, _, _ = forward(tok)
+                bd.bd_confidence_select("f32", B, H, V, h, h_prev, w["W"], bits, tau, sub_block,
+                                        tok, unmask, None, None, sel_ws)
             log.append(unmask.cpu().numpy().view(np.uint32).copy())
         h, k, v = forward(tok)       # the finished block with its final tokens
         bd.bd_cache_commit(cache, k, v, seq_ids, 1)
         h_prev = h[:, BLOCK - 1].contiguous()
         tokens_all.append(tok)
         unmasked.append(log)
-    return dict(tokens=torch.cat(tokens_all, dim=1).cpu().numpy(), steps=steps, unmasked=unmasked)
+    return dict(tokens=torch.cat(tokens_all, dim=1).cpu().numpy(), steps=steps, unmasked=unmasked,
+                refreshes=refreshes)
 
 
 def main():
@@ -140,19 +185,23 @@ def main():
     ap.add_argument("--blocks", type=int, default=4)
     ap.add_argument("--tau", type=float, default=0.9)
     ap.add_argument("--sub-block", type=int, default=8)
+    ap.add_argument("--dual-cache", action="store_true")
     args = ap.parse_args()
     model = TinyModel(TinyModelConfig())
     rng = np.random.default_rng(0)
     prompt = rng.integers(0, model.cfg.vocab, size=(args.batch, BLOCK * args.prompt_blocks))
-    decode(model, prompt.astype(np.int32), 1, args.tau, args.sub_block)  # warm-up
+    decode(model, prompt.astype(np.int32), 1, args.tau, args.sub_block,
+           dual_cache=args.dual_cache)  # warm-up
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    r = decode(model, prompt.astype(np.int32), args.blocks, args.tau, args.sub_block)
+    r = decode(model, prompt.astype(np.int32), args.blocks, args.tau, args.sub_block,
+               dual_cache=args.dual_cache)
     torch.cuda.synchronize()
     dt = time.perf_counter() - t0
     print(json.dumps({"tokens_per_s": args.batch * args.blocks * BLOCK / dt,
                       "mean_steps_per_block": float(r["steps"].mean()),
                       "tau": args.tau, "sub_block": args.sub_block, "batch": args.batch,
+                      "dual_cache": args.dual_cache, "refresh_steps": r["refreshes"],
                       "model": dataclasses.asdict(model.cfg)}))
 
 

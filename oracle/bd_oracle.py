@@ -53,6 +53,25 @@ R9  Masked-token cross-entropy of training ([N1] key design 2, the L_block
     row in its sequence and contributes nothing.  The equation's
     expectation is left to the caller: the step returns the per-position
     losses and their sum over the scored positions.
+R10 Decoding loop ([N1] "Overall framework" and key design 3; [N4]
+    "Acceleration engine" item 1): blocks of 32 are decoded left to right;
+    a block starts with every position [MASK]; each denoising step runs the
+    model on the block over the cache and applies the unmask rule (R7),
+    until no position is [MASK]; the finished block is run once more with
+    its final tokens and that run's K/V are committed to the cache, its last
+    hidden row being the next block's h_prev.  The model is a caller-given
+    single layer: x = E[token] (row V of E embeds [MASK]), q/k/v = x Wq /
+    Wk / Wv, h = x + attn(q, k, v) Wo, logits = W h.
+R11 Sub-block DualCache ([N1] key design 3; [N4] "Acceleration engine"
+    item 1: inside the block being decoded, the K/V of its prefix and
+    suffix are cached across the iterative refinement; [N1] "Limitations":
+    the reuse is approximate).  Per sequence, at the first step of each
+    active sub-block (R7) the whole block is run and its K, V and hidden
+    rows are cached (a refresh); at the following steps of that sub-block
+    only the active sub-block's S rows are fresh: the attention reads the
+    cached K/V for the other 32 - S rows, and the shifted hidden rows
+    outside the active sub-block are the cached ones.  With S = 32 the
+    active sub-block is the whole block, so the loop is the exact one.
 R8  Ambiguity: a position's token is ambiguous when its top-2 logit gap is
     < 1e-3; a sequence's unmask decision is ambiguous when some candidate has
     |p_max - tau| < 1e-4 (only for tau < 1: p_max = 1/Z with Z >= 1 never
@@ -76,6 +95,7 @@ __all__ = [
     "full_sequence_attn", "mixed_mask", "mask_attn", "shifted_rows",
     "lm_logits", "softmax_stats", "active_candidates", "select",
     "ambiguity", "confidence_select", "ce_positions", "masked_ce",
+    "MASK_TOKEN", "mask_bits", "decode_loop",
 ]
 
 
@@ -407,3 +427,120 @@ def masked_ce(h, W, targets, masked_bits, dtype: str = "f32", positions=None, ch
             loss[s, i] = lse[r] - logits[r, int(targets[s, i])]
     vals = np.array([loss[s, i] for s, i in pos], dtype=np.float64)
     return dict(loss=loss, total=float(vals.sum()), count=len(pos))
+
+
+# ----------------------------------------------------------------------------
+# the decoding loop, exact and with the sub-block DualCache (readings R10, R11)
+# ----------------------------------------------------------------------------
+MASK_TOKEN = -1  # id held by a still-masked position (outside [0, V))
+
+
+def mask_bits(tokens) -> np.ndarray:
+    """``[B, 32]`` tokens -> ``[B]`` words, bit i set where position i is [MASK]."""
+    tokens = np.asarray(tokens)
+    return np.array([sum(1 << i for i in range(BLOCK) if tokens[s, i] == MASK_TOKEN)
+                     for s in range(tokens.shape[0])], dtype=np.uint32)
+
+
+def decode_loop(weights, prompt, n_blocks: int, tau: float, sub_block: int, *,
+                n_heads_q: int, n_heads_kv: int, head_dim: int, rope_theta: float,
+                dual_cache: bool = False, trace: bool = False):
+    """Decode ``n_blocks`` blocks after ``prompt`` (``[B, 32 n]`` tokens) with
+    the single-layer model of reading R10, exactly or with the sub-block
+    DualCache of reading R11.
+
+    ``weights``: dict of float arrays E ``[V + 1, H]``, Wq ``[H, Hq d]``,
+    Wk / Wv ``[H, Hkv d]``, Wo ``[Hq d, H]``, W ``[V, H]``.  Returns dict
+    ``tokens`` ``[B, 32 (n + n_blocks)]``, ``steps`` ``[n_blocks, B]`` (steps
+    each sequence took per block), ``unmasked`` (per block, per step, the
+    ``[B]`` unmask words), ``ambiguous_at`` ((block, step) of the first
+    decision flagged by reading R8, or None).  With ``trace``, also
+    ``records``: per step (block, step, refresh flags ``[B]``, p_max of the
+    step, p_max of the exact step on the same tokens and cache).
+    """
+    E, Wq, Wk, Wv, Wo, W = (np.asarray(weights[n], np.float64)
+                            for n in ("E", "Wq", "Wk", "Wv", "Wo", "W"))
+    prompt = np.asarray(prompt)
+    B, P = prompt.shape
+    V = W.shape[0]
+    Hq, Hkv, d = n_heads_q, n_heads_kv, head_dim
+    cache = OracleCache(B, Hkv, d, rope_theta)
+
+    def project(tok):
+        x = E[np.where(tok == MASK_TOKEN, V, tok)]
+        return (x, (x @ Wq).reshape(B, BLOCK, Hq, d), (x @ Wk).reshape(B, BLOCK, Hkv, d),
+                (x @ Wv).reshape(B, BLOCK, Hkv, d))
+
+    def hidden(x, q, k, v):
+        return x + block_attn(cache, q, k, v).reshape(B, BLOCK, Hq * d) @ Wo
+
+    def commit(k, v):
+        for s in range(B):
+            cache.commit(s, k[s], v[s])
+
+    h_prev = np.zeros((B, E.shape[1]))
+    for b in range(P // BLOCK):  # the prompt, block by block
+        x, q, k, v = project(prompt[:, b * BLOCK:(b + 1) * BLOCK])
+        h = hidden(x, q, k, v)
+        commit(k, v)
+        h_prev = h[:, BLOCK - 1]
+    toks, logs, records = [prompt], [], []
+    steps = np.zeros((n_blocks, B), np.int64)
+    ambiguous_at = None
+    for b in range(n_blocks):
+        tok = np.full((B, BLOCK), MASK_TOKEN, np.int64)
+        log = []
+        cached_sub = [None] * B  # active sub-block the DualCache was filled for
+        Kc = np.zeros((B, BLOCK, Hkv, d))
+        Vc = np.zeros((B, BLOCK, Hkv, d))
+        Hc = np.zeros((B, BLOCK, E.shape[1]))
+        while (tok == MASK_TOKEN).any():
+            bits = mask_bits(tok)
+            steps[b] += (tok == MASK_TOKEN).any(axis=1)
+            x, q, k, v = project(tok)
+            refresh = np.ones(B, bool)
+            if dual_cache:
+                kb, vb = k.copy(), v.copy()
+                rows = np.zeros((B, BLOCK), bool)  # the active sub-block's rows
+                for s in range(B):
+                    first = min(i for i in range(BLOCK) if tok[s, i] == MASK_TOKEN) \
+                        if (tok[s] == MASK_TOKEN).any() else 0
+                    a = first // sub_block
+                    rows[s, a * sub_block:(a + 1) * sub_block] = True
+                    refresh[s] = cached_sub[s] != a
+                    if refresh[s]:
+                        Kc[s], Vc[s] = k[s], v[s]
+                        cached_sub[s] = a
+                    kb[s] = np.where(rows[s][:, None, None], k[s], Kc[s])
+                    vb[s] = np.where(rows[s][:, None, None], v[s], Vc[s])
+                h_new = hidden(x, q, kb, vb)
+                h = np.empty_like(h_new)
+                for s in range(B):
+                    if refresh[s]:
+                        Hc[s] = h_new[s]
+                    h[s] = np.where(rows[s][:, None], h_new[s], Hc[s])
+            else:
+                h = hidden(x, q, k, v)
+            r = confidence_select(h, h_prev, W, bits, tau, sub_block, tok, "f32")
+            if trace:
+                exact = r if not dual_cache else confidence_select(
+                    hidden(x, q, k, v), h_prev, W, bits, tau, sub_block, tok, "f32")
+                records.append(dict(block=b, step=len(log), refresh=refresh.copy(),
+                                    pmax=r["pmax"], pmax_exact=exact["pmax"]))
+            picked_amb = any(r["token_ambiguous"][s, i] for s in range(B) for i in range(BLOCK)
+                             if (int(r["unmask"][s]) >> i) & 1)
+            if ambiguous_at is None and (r["decision_ambiguous"].any() or picked_amb):
+                ambiguous_at = (b, len(log))
+            tok = r["tokens"].astype(np.int64)
+            log.append(r["unmask"].astype(np.uint32))
+        x, q, k, v = project(tok)  # the finished block with its final tokens
+        h = hidden(x, q, k, v)
+        commit(k, v)
+        h_prev = h[:, BLOCK - 1]
+        toks.append(tok)
+        logs.append(log)
+    out = dict(tokens=np.concatenate(toks, 1), steps=steps, unmasked=logs,
+               ambiguous_at=ambiguous_at)
+    if trace:
+        out["records"] = records
+    return out

@@ -21,54 +21,31 @@ def _cuda():
     from decoding_bd_block_b200 import bd  # noqa: F401  (fails loudly if libbd.so is missing)
 
 
-def oracle_decode(model, prompt, n_blocks, tau, S):
-    """The loop of decode.decode in float64 on the oracle's attention and select."""
-    from decoding_bd_block_b200.workloads import BLOCK, MASK_TOKEN
+def oracle_decode(model, prompt, n_blocks, tau, S, dual_cache=False):
+    """The loop of decode.decode in float64 on the oracle (reading R10; R11
+    with ``dual_cache``)."""
     c = model.cfg
-    B, P = prompt.shape
-    Hq, Hkv, d, V = c.n_heads_q, c.n_heads_kv, c.head_dim, c.vocab
-    E, Wq, Wk, Wv, Wo = (getattr(model, n).astype(np.float64) for n in ("E", "Wq", "Wk", "Wv", "Wo"))
-    cache = O.OracleCache(B, Hkv, d, c.rope_theta)
+    weights = {n: getattr(model, n) for n in ("E", "Wq", "Wk", "Wv", "Wo", "W")}
+    return O.decode_loop(weights, prompt, n_blocks, tau, S, n_heads_q=c.n_heads_q,
+                         n_heads_kv=c.n_heads_kv, head_dim=c.head_dim, rope_theta=c.rope_theta,
+                         dual_cache=dual_cache)
 
-    def forward(tok):
-        x = E[np.where(tok == MASK_TOKEN, V, tok)]
-        q, k, v = (x @ Wq).reshape(B, BLOCK, Hq, d), (x @ Wk).reshape(B, BLOCK, Hkv, d), \
-            (x @ Wv).reshape(B, BLOCK, Hkv, d)
-        att = O.block_attn(cache, q, k, v)
-        return x + att.reshape(B, BLOCK, Hq * d) @ Wo, k, v
 
-    def commit(k, v):
-        for s in range(B):
-            cache.commit(s, k[s], v[s])
-
-    h_prev = np.zeros((B, c.hidden))
-    for b in range(P // BLOCK):
-        h, k, v = forward(prompt[:, b * BLOCK:(b + 1) * BLOCK])
-        commit(k, v)
-        h_prev = h[:, BLOCK - 1]
-    toks, steps, logs, ambiguous_at = [prompt], np.zeros((n_blocks, B), np.int64), [], None
-    for b in range(n_blocks):
-        tok = np.full((B, BLOCK), MASK_TOKEN, np.int32)
-        log = []
-        while (tok == MASK_TOKEN).any():
-            bits = np.array([sum(1 << i for i in range(BLOCK) if tok[s, i] == MASK_TOKEN)
-                             for s in range(B)], dtype=np.uint32)
-            steps[b] += (tok == MASK_TOKEN).any(axis=1)
-            h, _, _ = forward(tok)
-            r = O.confidence_select(h, h_prev, model.W, bits, tau, S, tok, "f32")
-            picked_amb = any(r["token_ambiguous"][s, i] for s in range(B) for i in range(BLOCK)
-                             if (int(r["unmask"][s]) >> i) & 1)
-            if ambiguous_at is None and (r["decision_ambiguous"].any() or picked_amb):
-                ambiguous_at = (b, len(log))
-            tok = r["tokens"].astype(np.int32)
-            log.append(r["unmask"].astype(np.uint32))
-        h, k, v = forward(tok)
-        commit(k, v)
-        h_prev = h[:, BLOCK - 1]
-        toks.append(tok)
-        logs.append(log)
-    return dict(tokens=np.concatenate(toks, 1), steps=steps, unmasked=logs,
-                ambiguous_at=ambiguous_at)
+def check_against_oracle(got, ref):
+    """Every token, step count and unmask word equal, up to the first decision
+    the oracle flags as ambiguous (which must not come too early)."""
+    assert ref["ambiguous_at"] is None or ref["ambiguous_at"] >= (0, 8)
+    if ref["ambiguous_at"] is None:
+        assert np.array_equal(got["tokens"], ref["tokens"])
+        assert np.array_equal(got["steps"], ref["steps"])
+        for a, b in zip(got["unmasked"], ref["unmasked"]):
+            assert len(a) == len(b) and all(np.array_equal(x, y) for x, y in zip(a, b))
+    else:                                                      # equal up to the flagged step
+        b0, j0 = ref["ambiguous_at"]
+        for b in range(b0):
+            assert all(np.array_equal(x, y) for x, y in zip(got["unmasked"][b], ref["unmasked"][b]))
+        assert all(np.array_equal(x, y)
+                   for x, y in zip(got["unmasked"][b0][:j0], ref["unmasked"][b0][:j0]))
 
 
 @pytest.mark.parametrize("tau,S", [(1.0, 8), (0.9, 8), (0.5, 32)])
@@ -87,16 +64,22 @@ def test_decode_loop_matches_oracle_loop(tau, S):
                 assert all(bin(int(x)).count("1") == 1 for x in u)
     print("tau", tau, "S", S, "steps", got["steps"].tolist(), "oracle ambiguous at",
           ref["ambiguous_at"])
-    # the model must be decisive enough for the comparison to mean something
-    assert ref["ambiguous_at"] is None or ref["ambiguous_at"] >= (0, 8)
-    if ref["ambiguous_at"] is None:
-        assert np.array_equal(got["tokens"], ref["tokens"])
-        assert np.array_equal(got["steps"], ref["steps"])
-        for a, b in zip(got["unmasked"], ref["unmasked"]):
-            assert len(a) == len(b) and all(np.array_equal(x, y) for x, y in zip(a, b))
-    else:                                                      # equal up to the flagged step
-        b0, j0 = ref["ambiguous_at"]
-        for b in range(b0):
-            assert all(np.array_equal(x, y) for x, y in zip(got["unmasked"][b], ref["unmasked"][b]))
-        assert all(np.array_equal(x, y)
-                   for x, y in zip(got["unmasked"][b0][:j0], ref["unmasked"][b0][:j0]))
+    check_against_oracle(got, ref)
+
+
+@pytest.mark.parametrize("tau,S", [(0.9, 8), (1.0, 8), (0.9, 16)])
+def test_decode_loop_dual_cache_matches_oracle_loop(tau, S):
+    """The sub-block DualCache loop against the oracle's DualCache loop: the
+    cache is approximate, so the reference is the oracle's own definition."""
+    from decoding_bd_block_b200.decode import TinyModel, TinyModelConfig, decode
+    model = TinyModel(TinyModelConfig())
+    rng = np.random.default_rng(12)
+    prompt = rng.integers(0, model.cfg.vocab, size=(2, 64)).astype(np.int32)
+    got = decode(model, prompt, n_blocks=2, tau=tau, sub_block=S, dual_cache=True)
+    ref = oracle_decode(model, prompt, 2, tau, S, dual_cache=True)
+    assert (got["steps"] >= 32 // S).all() and (got["steps"] <= 32).all()
+    # every sequence refreshes once per sub-block and block
+    assert got["refreshes"] == 2 * 2 * (32 // S)
+    print("dual cache: tau", tau, "S", S, "steps", got["steps"].tolist(), "oracle ambiguous at",
+          ref["ambiguous_at"])
+    check_against_oracle(got, ref)
