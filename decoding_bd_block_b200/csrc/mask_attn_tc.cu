@@ -88,9 +88,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint8_t kv_kind[64];   // 1: partial, 2: full
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // Heaviest query tiles first: clean tiles late in the sequence see the most keys.
-  const int qt = a.n_qt - 1 - static_cast<int>(blockIdx.x);
-  const int pr = blockIdx.y, n = blockIdx.z;
+  // Heaviest query tiles first over the whole grid (blockIdx.z, the
+  // slowest-varying index, is the work rank): noisy query tile w and clean
+  // query tile n_qt / 2 + w both see w + 1 key tiles, so the ranks take
+  // them in pairs from the last w down.
+  const int half = a.n_qt / 2, rank = blockIdx.z, wq = half - 1 - rank / 2;
+  const int qt = (rank & 1) ? wq : half + wq;
+  const int pr = blockIdx.x, n = blockIdx.y;
   const int g = pr / a.per_group;
   const int w = pr % a.per_group;
   const int h0 = g * a.G + 2 * w;                 // first head of the pair
@@ -378,7 +382,7 @@ cudaError_t launch_mask_attn_tc(const bd_attn_shape& sh, const void* q, const vo
   cudaFuncSetAttribute(mask_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        kSmemBytes);
   a.per_group = (a.G + 1) / 2;
-  mask_attn_tc_kernel<<<dim3(a.n_qt, a.per_group * Hkv, n_seqs), kThreads, kSmemBytes, st>>>(
+  mask_attn_tc_kernel<<<dim3(a.per_group * Hkv, n_seqs, a.n_qt), kThreads, kSmemBytes, st>>>(
       tm_q, tm_k, tm_v, a);
   count_launches(1);
   return cudaGetLastError();
