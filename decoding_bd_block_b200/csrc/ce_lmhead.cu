@@ -12,8 +12,8 @@
 //     (32 KB): 64 KB for two 128 x 256 x 64 products.
 //   * persistent CTAs, one per SM, take units u = blockIdx.x + k * gridDim.x
 //     with rp fastest, so the CTAs running at one time stream the same few
-//     vocab ranges: W comes from HBM about once, the rows (they fit in L2)
-//     from L2.
+//     vocab ranges: W comes from HBM a few times in all (CTAs drift apart
+//     over a range), the rows (they fit in L2) from L2.
 //   * warp 0 streams the stages by TMA (3 stages), warp 1 issues tcgen05.mma
 //     into two 256-column TMEM accumulators (one per row tile), warps 2-17
 //     each drain 32 rows x 128 columns after a W tile; a thread owns one row,
