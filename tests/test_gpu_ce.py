@@ -90,6 +90,16 @@ def test_masked_ce_nothing_scored_and_bad_target():
     assert not np.isnan(np.delete(loss[0], [0, 5])).any()
 
 
+def test_masked_ce_rows_path_nothing_scored():
+    """>= 2048 packed rows allocated (the rows-as-M LM head) but no position
+    scored: no unit of work, count 0, sum 0, every loss NaN."""
+    cfg = dataclasses.replace(W.MASKED_CE, samples=2, L=1024, hidden=264, vocab=20001, seed=207)
+    d = W.make_ce_inputs(cfg)
+    d0 = dict(d, masked_bits=np.zeros_like(d["masked_bits"]))
+    loss, total, count = _run(cfg, d0)
+    assert count == 0 and total == 0.0 and np.isnan(loss).all()
+
+
 def test_masked_ce_full_size_sampled_and_deterministic():
     cfg = W.MASKED_CE
     d = W.make_ce_inputs(cfg)
