@@ -215,17 +215,30 @@ def source_sha(paths):
 # --------------------------------------------------------------------------
 # the oracle as a CPU baseline (test infrastructure, timed as it stands)
 # --------------------------------------------------------------------------
-def oracle_step_sample(cfg, a_in, s_in, frac: float, tau: float, S: int):
-    """One oracle step on a bounded sample: full block attention, and the
-    LM-head statistics / selection over the first `frac` of the vocabulary.
-    Returns the masked-position equivalents scored (frac x masked positions)."""
+def oracle_caches(cfg, a_in, seqs=None):
+    """The oracle's cache (prefix K rotated at commit) of the given sequences:
+    built once, outside any timed region, as the GPU arm's cache is."""
+    import oracle as O
+    seqs = range(cfg.batch) if seqs is None else seqs
+    out = {}
+    for s in seqs:
+        c = O.OracleCache(1, cfg.n_heads_kv, cfg.head_dim, cfg.rope_theta)
+        if a_in["prefix_len"][s]:
+            c.commit(0, O.widen(a_in["prefix_k"][s], cfg.dtype),
+                     O.widen(a_in["prefix_v"][s], cfg.dtype))
+        out[s] = c
+    return out
+
+
+def oracle_step_sample(cfg, a_in, s_in, frac: float, tau: float, S: int, caches=None):
+    """One oracle step on a bounded sample: block attention of the sequences
+    in ``caches`` (all of them when None), and the LM-head statistics /
+    selection over the first `frac` of the vocabulary.  Returns the
+    masked-position equivalents scored (frac x masked positions)."""
     import oracle as O
     if a_in is not None:
-        for s in range(cfg.batch):
-            c = O.OracleCache(1, cfg.n_heads_kv, cfg.head_dim, cfg.rope_theta)
-            if a_in["prefix_len"][s]:
-                c.commit(0, O.widen(a_in["prefix_k"][s], cfg.dtype),
-                         O.widen(a_in["prefix_v"][s], cfg.dtype))
+        caches = oracle_caches(cfg, a_in) if caches is None else caches
+        for s, c in caches.items():
             O.block_attn_seq(c.k[0], c.v[0], O.widen(a_in["q"][s], cfg.dtype),
                              O.widen(a_in["k_blk"][s], cfg.dtype),
                              O.widen(a_in["v_blk"][s], cfg.dtype), cfg.rope_theta)
@@ -248,14 +261,15 @@ def blas_threads():
 
 def cpu_baseline(cfg, a_in, s_in, tau, S, budget_s):
     """Time the oracle on a sample of the workload for about `budget_s`."""
+    caches = oracle_caches(cfg, a_in) if a_in is not None else None
     t0 = time.perf_counter()
-    oracle_step_sample(cfg, a_in, s_in, 0.02, tau, S)       # probe: 2% of the vocab
+    oracle_step_sample(cfg, a_in, s_in, 0.02, tau, S, caches)  # probe: 2% of the vocab
     probe = max(time.perf_counter() - t0, 1e-3)
     frac = float(min(1.0, max(0.02, 0.02 * budget_s / probe / 2)))
     scored, t_total, n = 0.0, 0.0, 0
     while t_total < budget_s * 0.5 or n == 0:
         t0 = time.perf_counter()
-        scored += oracle_step_sample(cfg, a_in, s_in, frac, tau, S)
+        scored += oracle_step_sample(cfg, a_in, s_in, frac, tau, S, caches)
         t_total += time.perf_counter() - t0
         n += 1
     import platform
@@ -270,40 +284,137 @@ def cpu_baseline(cfg, a_in, s_in, tau, S, budget_s):
 # --------------------------------------------------------------------------
 # arms
 # --------------------------------------------------------------------------
+def reference_line(args, cfg_name, metric, unit, value, t, config, sample):
+    """The JSON line of the reference arm (the oracle, timed on the host)."""
+    return {
+        "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference", "config": dict(workload=cfg_name, **config),
+        "cpu_baseline": {"value": value, "unit": unit, "kind": "oracle", "cores": blas_threads(),
+                         "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def reference_budget(args):
+    """Seconds of oracle work per step, so that the whole run ends in a few minutes."""
+    return 150.0 / max(1, args.steps + args.warmup)
+
+
 def run_reference(args, cfg, tau, S):
     a_in = W.make_attn_inputs(cfg)
     s_in = W.make_select_inputs(cfg) if cfg.hidden else None
-    if s_in is not None:
-        s_in["n_scored"] = int(sum(bin(int(b)).count("1") for b in s_in["masked_bits"]))
+    if s_in is None:  # attention only: a bounded number of whole sequences per step
+        caches = oracle_caches(cfg, a_in, [0])
+        t0 = time.perf_counter()
+        oracle_step_sample(cfg, a_in, None, 0.0, tau, S, caches)
+        probe = max(time.perf_counter() - t0, 1e-3)
+        n_seq = int(min(cfg.batch, max(1, reference_budget(args) // probe)))
+        caches = oracle_caches(cfg, a_in, range(n_seq))
+        for _ in range(args.warmup):
+            oracle_step_sample(cfg, a_in, None, 0.0, tau, S, caches)
+        t = 0.0
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            oracle_step_sample(cfg, a_in, None, 0.0, tau, S, caches)
+            t += time.perf_counter() - t0
+        rows = n_seq * W.BLOCK * cfg.n_heads_q * args.steps
+        line = reference_line(
+            args, cfg.name, "query rows attended/s per denoise step (block attention only)",
+            "query rows/s", rows / t, t, {"batch": cfg.batch, "sequences_per_step": n_seq},
+            f"each step: the block attention of {n_seq} of the {cfg.batch} sequences of workload "
+            f"{cfg.name} (the cache rotated once, before timing)")
+        print(json.dumps(line), flush=True)
+        return
+    s_in["n_scored"] = int(sum(bin(int(b)).count("1") for b in s_in["masked_bits"]))
+    caches = oracle_caches(cfg, a_in)
     t0 = time.perf_counter()
-    oracle_step_sample(cfg, a_in, s_in, 0.02, tau, S)
+    oracle_step_sample(cfg, a_in, s_in, 0.02, tau, S, caches)
     probe = max(time.perf_counter() - t0, 1e-3)
-    per_step_budget = 150.0 / max(1, args.steps + args.warmup)
-    frac = float(min(1.0, max(0.002, 0.02 * per_step_budget / probe)))
+    frac = float(min(1.0, max(0.002, 0.02 * reference_budget(args) / probe)))
     for _ in range(args.warmup):
-        oracle_step_sample(cfg, a_in, s_in, frac, tau, S)
+        oracle_step_sample(cfg, a_in, s_in, frac, tau, S, caches)
     scored, t = 0.0, 0.0
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        scored += oracle_step_sample(cfg, a_in, s_in, frac, tau, S)
+        scored += oracle_step_sample(cfg, a_in, s_in, frac, tau, S, caches)
         t += time.perf_counter() - t0
-    value = scored / t
-    line = {
-        "metric": "masked positions scored/s per denoise step", "value": value,
-        "unit": "masked positions scored/s", "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "impl": "reference",
-        "config": {"workload": cfg.name, "batch": cfg.batch, "tau": tau, "sub_block": S,
-                   "vocab_fraction_per_step": frac},
-        "cpu_baseline": {"value": value, "unit": "masked positions scored/s", "kind": "oracle",
-                         "cores": blas_threads(),
-                         "sample": f"each step: full block attention + LM-head statistics over "
-                                   f"{frac:.2%} of the vocabulary of workload {cfg.name}"},
-        "e2e": {"value": value, "unit": "masked positions scored/s", "h2d_bytes_per_step": 0,
-                "d2h_bytes_per_step": 0},
-    }
+    line = reference_line(
+        args, cfg.name, "masked positions scored/s per denoise step", "masked positions scored/s",
+        scored / t, t, {"batch": cfg.batch, "tau": tau, "sub_block": S,
+                        "vocab_fraction_per_step": frac},
+        f"each step: full block attention + LM-head statistics over {frac:.2%} of the "
+        f"vocabulary of workload {cfg.name}")
     print(json.dumps(line), flush=True)
+
+
+def run_reference_mask_attn(args, cfg):
+    """The oracle's 2L x 2L masked attention on a bounded sample of query rows."""
+    import oracle as O
+    t = W.make_mask_attn_inputs(cfg)
+    q, k, v = (O.widen(t[x], cfg.dtype) for x in ("q", "k", "v"))
+    rng = np.random.default_rng(0)
+    per = probe_cost(lambda n: O.mask_attn(q, k, v, cfg.L, cfg.block, rows=np.arange(n)),
+                     16)  # per query row over all views
+    n_rows = int(min(2 * cfg.L, max(8, 0.5 * reference_budget(args) / per)))  # half: margin
+    rows = np.sort(rng.choice(2 * cfg.L, n_rows, replace=False))
+    for _ in range(args.warmup):
+        O.mask_attn(q, k, v, cfg.L, cfg.block, rows=rows)
+    tt = 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        O.mask_attn(q, k, v, cfg.L, cfg.block, rows=rows)
+        tt += time.perf_counter() - t0
+    units = n_rows * cfg.n_seqs * cfg.n_heads_q * args.steps
+    line = reference_line(
+        args, cfg.name, "query rows attended/s (2L x 2L complementary-mask attention)",
+        "query rows/s", units / tt, tt,
+        {"views": cfg.n_seqs, "L": cfg.L, "block": cfg.block, "rows_per_view_per_step": n_rows},
+        f"each step: {n_rows} of the {2 * cfg.L} query rows (all heads) of each of the "
+        f"{cfg.n_seqs} views of workload {cfg.name}")
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_ce(args, cfg):
+    """The oracle's masked cross-entropy on a bounded sample of scored positions."""
+    import oracle as O
+    d = W.make_ce_inputs(cfg)
+    pos = O.ce_positions(d["masked_bits"])
+    per = probe_cost(lambda n: O.masked_ce(d["h"], d["W"], d["targets"], d["masked_bits"],
+                                           cfg.dtype, positions=pos[:n]), 256)
+    # whole chunks of 256 positions (the oracle's unit of work)
+    n_pos = int(min(len(pos), max(256, 0.5 * reference_budget(args) / per // 256 * 256)))
+    rng = np.random.default_rng(0)
+    sample = [pos[i] for i in sorted(rng.choice(len(pos), n_pos, replace=False))]
+    for _ in range(args.warmup):
+        O.masked_ce(d["h"], d["W"], d["targets"], d["masked_bits"], cfg.dtype, positions=sample)
+    tt = 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        O.masked_ce(d["h"], d["W"], d["targets"], d["masked_bits"], cfg.dtype, positions=sample)
+        tt += time.perf_counter() - t0
+    line = reference_line(
+        args, cfg.name, "masked positions' cross-entropy computed/s (training batch)",
+        "scored positions/s", n_pos * args.steps / tt, tt,
+        {"sequences": cfg.n_seqs, "L": cfg.L, "hidden": cfg.hidden, "vocab": cfg.vocab,
+         "positions_per_step": n_pos},
+        f"each step: the loss at {n_pos} of the {len(pos)} scored positions of workload {cfg.name}")
+    print(json.dumps(line), flush=True)
+
+
+def probe_cost(fn, n: int):
+    """Seconds per unit of fn(n), fixed costs included (so a sample sized by it
+    stays within its budget): one untimed call to warm up, one timed."""
+    fn(n)
+    t0 = time.perf_counter()
+    fn(n)
+    return max((time.perf_counter() - t0) / n, 1e-6)
+
+
+def reference_rank0():
+    """Under torchrun the reference arm runs on rank 0 only."""
+    return int(os.environ.get("RANK", "0")) == 0
 
 
 def run_ours(args, cfg, tau, S, dist: Dist):
@@ -643,8 +754,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.workload == W.MASK_ATTN.name:
         if args.impl == "reference":
-            print(json.dumps({"impl": "reference", "unavailable":
-                              "the reference arm times the decoding-step workloads only"}))
+            if reference_rank0():
+                run_reference_mask_attn(args, W.MASK_ATTN)
             return 0
         dist = Dist("nccl")
         try:
@@ -654,8 +765,8 @@ def main(argv=None):
         return 0
     if args.workload == W.MASKED_CE.name:
         if args.impl == "reference":
-            print(json.dumps({"impl": "reference", "unavailable":
-                              "the reference arm times the decoding-step workloads only"}))
+            if reference_rank0():
+                run_reference_ce(args, W.MASKED_CE)
             return 0
         dist = Dist("nccl")
         try:
@@ -667,11 +778,8 @@ def main(argv=None):
     tau = args.tau if args.tau is not None else cfg.taus[0]
     S = args.sub_block if args.sub_block is not None else cfg.sub_block
     if args.impl == "reference":
-        world = int(os.environ.get("WORLD_SIZE", "1"))
-        rank = int(os.environ.get("RANK", "0"))
-        if world > 1 and rank != 0:
-            return 0
-        run_reference(args, cfg, tau, S)
+        if reference_rank0():
+            run_reference(args, cfg, tau, S)
         return 0
     dist = Dist("nccl")
     try:
