@@ -5,6 +5,8 @@
 #include <cstring>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "bd_common.cuh"
 
 namespace bd {
@@ -18,6 +20,15 @@ void rope_freq_table(int d, double theta, RopeFreq* f) {
 }  // namespace bd
 
 namespace {
+
+// A profiler-visible range named after the entry point, for the duration of
+// the call (NVTX: a no-op unless a tool such as Nsight is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 thread_local char g_cuda_err[256] = "";
 
@@ -82,6 +93,7 @@ long long bd_kernel_launches(void) { return bd::g_launches.load(std::memory_orde
 
 int bd_cache_commit(const bd_attn_shape* sh, bd_kv_cache* c, const void* k, const void* v,
                     const int32_t* seq_ids, int32_t n_seqs, int32_t n_new_blocks, void* stream) {
+  NvtxRange nvtx_range("bd_cache_commit");
   int st = check_shape(sh);
   if (st) return st;
   if ((st = check_cache(sh, c))) return st;
@@ -142,6 +154,7 @@ int bd_block_attn_workspace_size(const bd_attn_shape* sh, const bd_kv_cache* c, 
 
 int bd_block_attn(const bd_attn_shape* sh, const bd_kv_cache* c, const void* q, const void* k,
                   const void* v, void* out, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("bd_block_attn");
   int st = check_shape(sh);
   if (st) return st;
   if ((st = check_cache(sh, c))) return st;
@@ -195,6 +208,7 @@ int bd_confidence_select(int32_t dtype, int32_t batch, int32_t hidden, int32_t v
                          const uint32_t* masked_bits, float tau, int32_t sub_block,
                          int32_t* tokens, uint32_t* unmask_bits, float* pmax_out,
                          int32_t* argmax_out, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("bd_confidence_select");
   return confidence_select(dtype, batch, hidden, vocab, h, h_prev, w, masked_bits, tau, sub_block,
                            tokens, unmask_bits, pmax_out, argmax_out, ws, ws_bytes, stream, 0);
 }
@@ -204,6 +218,7 @@ int bd_confidence_select_active(int32_t dtype, int32_t batch, int32_t hidden, in
                                 const uint32_t* masked_bits, float tau, int32_t sub_block,
                                 int32_t* tokens, uint32_t* unmask_bits, float* pmax_out,
                                 int32_t* argmax_out, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("bd_confidence_select_active");
   return confidence_select(dtype, batch, hidden, vocab, h, h_prev, w, masked_bits, tau, sub_block,
                            tokens, unmask_bits, pmax_out, argmax_out, ws, ws_bytes, stream, 1);
 }
@@ -222,6 +237,7 @@ int bd_masked_ce(int32_t dtype, int32_t n_seqs, int32_t seq_len, int32_t hidden,
                  const void* h, const void* w, const int32_t* targets,
                  const uint32_t* masked_bits, float* loss_out, float* loss_sum, int32_t* n_scored,
                  void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("bd_masked_ce");
   if (n_seqs <= 0 || seq_len <= 0 || hidden <= 0 || vocab <= 0) return BD_ERR_INVALID_ARG;
   if (dtype != BD_F32 && dtype != BD_BF16) return BD_ERR_UNSUPPORTED;
   if (seq_len % bd::kBlock != 0 || hidden % 8 != 0) return BD_ERR_UNSUPPORTED;
@@ -240,6 +256,7 @@ int bd_masked_ce(int32_t dtype, int32_t n_seqs, int32_t seq_len, int32_t hidden,
 
 int bd_block_mask_attn(const bd_attn_shape* sh, const void* q, const void* k, const void* v,
                        void* out, int32_t n_seqs, int32_t L, int32_t block, void* stream) {
+  NvtxRange nvtx_range("bd_block_mask_attn");
   int st = check_shape(sh);
   if (st) return st;
   if (!q || !k || !v || !out || n_seqs <= 0 || n_seqs > 65535 || L <= 0 || block <= 0)

@@ -17,6 +17,8 @@
 // cudaGetSymbolAddress, with that device current, and cached.
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "bd_common.cuh"
 
 namespace bd {
@@ -51,12 +53,11 @@ void* scratch_for_current_device(cudaError_t* err) {
 }  // namespace
 }  // namespace bd
 
-extern "C" int bd_confidence_select_noalloc(int32_t dtype, int32_t batch, int32_t hidden,
-                                            int32_t vocab, const void* h, const void* h_prev,
-                                            const void* w, const uint32_t* masked_bits,
-                                            float tau, int32_t sub_block, int32_t* tokens,
-                                            uint32_t* unmask_bits, float* pmax_out,
-                                            int32_t* argmax_out, void* stream) {
+static int noalloc_call(int32_t dtype, int32_t batch, int32_t hidden, int32_t vocab,
+                        const void* h, const void* h_prev, const void* w,
+                        const uint32_t* masked_bits, float tau, int32_t sub_block,
+                        int32_t* tokens, uint32_t* unmask_bits, float* pmax_out,
+                        int32_t* argmax_out, void* stream) {
   if (batch <= 0 || batch > 65535 || hidden <= 0 || vocab <= 0) return BD_ERR_INVALID_ARG;
   if (dtype != BD_F32 && dtype != BD_BF16) return BD_ERR_UNSUPPORTED;
   // The scratch layout is the one bd_confidence_select asks its caller for;
@@ -71,3 +72,17 @@ extern "C" int bd_confidence_select_noalloc(int32_t dtype, int32_t batch, int32_
                               sub_block, tokens, unmask_bits, pmax_out, argmax_out, scratch,
                               static_cast<size_t>(BD_NOALLOC_SCRATCH_BYTES), stream);
 }
+
+extern "C" int bd_confidence_select_noalloc(int32_t dtype, int32_t batch, int32_t hidden,
+                                            int32_t vocab, const void* h, const void* h_prev,
+                                            const void* w, const uint32_t* masked_bits,
+                                            float tau, int32_t sub_block, int32_t* tokens,
+                                            uint32_t* unmask_bits, float* pmax_out,
+                                            int32_t* argmax_out, void* stream) {
+  nvtxRangePushA("bd_confidence_select_noalloc");
+  const int st = noalloc_call(dtype, batch, hidden, vocab, h, h_prev, w, masked_bits, tau, sub_block,
+                              tokens, unmask_bits, pmax_out, argmax_out, stream);
+  nvtxRangePop();
+  return st;
+}
+
