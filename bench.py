@@ -33,7 +33,7 @@ sys.path.insert(0, ROOT)
 
 from decoding_bd_block_b200 import workloads as W  # noqa: E402
 
-DEFAULT_WORKLOAD = W.QWEN15B_STEP.name
+DEFAULT_WORKLOAD = W.QWEN7B_RAGGED.name
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 SELECT_KERNEL_SOURCES = ("decoding_bd_block_b200/csrc/select_tc.cu", "decoding_bd_block_b200/csrc/tc_common.cuh")
@@ -259,12 +259,35 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(cfg, a_in, s_in, tau, S, budget_s):
-    """Time the oracle on a sample of the workload for about `budget_s`."""
+def cpu_baseline(cfg, a_in, s_in, tau, S, budget_s, got=None):
+    """Time the oracle on the host on a bounded sample of the workload, and,
+    when that sample is the whole step, compare the timed step's GPU outputs
+    (``got``) with it.  Returns (cpu_baseline dict, parity dict or None).
+
+    The sample is one whole oracle step (every sequence's block attention,
+    the LM head over the full vocabulary, the selection) when a 2% probe
+    predicts it fits in 3 x budget_s; otherwise a vocabulary fraction of the
+    step sized to about budget_s, and no parity block."""
+    import platform
     caches = oracle_caches(cfg, a_in) if a_in is not None else None
     t0 = time.perf_counter()
     oracle_step_sample(cfg, a_in, s_in, 0.02, tau, S, caches)  # probe: 2% of the vocab
     probe = max(time.perf_counter() - t0, 1e-3)
+    cpu = platform.processor() or platform.machine()
+    n_pos = s_in["n_scored"] if s_in else 0
+    if s_in is None or probe * 50 <= 3 * budget_s:  # (attention only: the probe was a whole step)
+        t0 = time.perf_counter()
+        ref = oracle_full_step(cfg, a_in, s_in, tau, S, caches)
+        t = time.perf_counter() - t0
+        base = {"value": (n_pos if s_in else cfg.batch * W.BLOCK * cfg.n_heads_q) / t,
+                "unit": "masked positions scored/s" if s_in else "query rows/s",
+                "cores": blas_threads(), "kind": "oracle",
+                "sample": (f"one whole oracle step of workload {cfg.name}: block attention of all "
+                           f"{cfg.batch} sequences"
+                           + (f" + LM-head statistics over the full vocabulary and selection "
+                              f"({n_pos} masked positions)" if s_in else "")
+                           + f"; fp64 numpy on {cpu}")}
+        return base, (parity_block(cfg, ref, got, tau, S) if got is not None else None)
     frac = float(min(1.0, max(0.02, 0.02 * budget_s / probe / 2)))
     scored, t_total, n = 0.0, 0.0, 0
     while t_total < budget_s * 0.5 or n == 0:
@@ -272,13 +295,78 @@ def cpu_baseline(cfg, a_in, s_in, tau, S, budget_s):
         scored += oracle_step_sample(cfg, a_in, s_in, frac, tau, S, caches)
         t_total += time.perf_counter() - t0
         n += 1
-    import platform
     return {"value": scored / t_total, "unit": "masked positions scored/s", "cores": blas_threads(),
             "kind": "oracle",
             "sample": (f"{n} oracle step(s) of workload {cfg.name}: full block attention + "
                        f"LM-head statistics and selection over {frac:.1%} of the vocabulary "
-                       f"({frac:.3f} x {s_in['n_scored'] if s_in else 0} masked positions per step); "
-                       f"fp64 numpy on {platform.processor() or platform.machine()}")}
+                       f"({frac:.3f} x {n_pos} masked positions per step); fp64 numpy on {cpu}")}, None
+
+
+def oracle_full_step(cfg, a_in, s_in, tau, S, caches):
+    """The oracle on the whole step: {s: block attention [32, Hq, d]} and the
+    selection result of the full vocabulary (None without a select part)."""
+    import oracle as O
+    attn = {}
+    if a_in is not None:
+        for s, c in caches.items():
+            attn[s] = O.block_attn_seq(c.k[0], c.v[0], O.widen(a_in["q"][s], cfg.dtype),
+                                       O.widen(a_in["k_blk"][s], cfg.dtype),
+                                       O.widen(a_in["v_blk"][s], cfg.dtype), cfg.rope_theta)
+    sel = None
+    if s_in is not None:
+        sel = O.confidence_select(s_in["h"], s_in["h_prev"], s_in["W"], s_in["masked_bits"], tau, S,
+                                  s_in["tokens"], cfg.dtype)
+    return attn, sel
+
+
+ATTN_TOL = {"f32": 1e-5, "bf16": 2e-2}  # max-abs bound of the attention outputs per storage type
+PMAX_TOL = 1e-4                          # p_max agreement the threshold band needs
+
+
+def parity_block(cfg, ref, got, tau, S):
+    """The timed step's GPU outputs against the oracle's whole step.
+
+    Decisions (unmask words) and tokens must be identical outside the
+    positions the oracle flags as ambiguous; the flagged ones are counted.
+    Attention: max-abs error against the oracle, with the stated bound."""
+    attn_ref, sel = ref
+    out = {"tau": tau, "sub_block": S}
+    ok = True
+    if attn_ref:
+        err = max(float(np.abs(got["out"][s] - attn_ref[s]).max()) for s in attn_ref)
+        out.update(attn_max_abs_err=err, attn_tol=ATTN_TOL[cfg.dtype],
+                   attn_sequences=len(attn_ref))
+        ok &= err <= ATTN_TOL[cfg.dtype]
+    if sel is not None:
+        bits = np.asarray(got["masked"], np.uint32)
+        pos = dec = tok = 0
+        bad_dec = bad_tok = bad_pmax = 0
+        pmax_err = 0.0
+        for s in range(len(bits)):
+            b = int(bits[s])
+            for i in range(W.BLOCK):
+                if not (b >> i) & 1:
+                    continue
+                pos += 1
+                pmax_err = max(pmax_err, abs(float(got["pmax"][s, i]) - float(sel["pmax"][s, i])))
+                bad_pmax += abs(float(got["pmax"][s, i]) - float(sel["pmax"][s, i])) > PMAX_TOL
+                if not sel["token_ambiguous"][s, i]:
+                    bad_tok += int(got["argmax"][s, i]) != int(sel["argmax"][s, i])
+            if sel["decision_ambiguous"][s]:
+                continue
+            dec += 1
+            bad_dec += int(got["unmask"][s]) != int(sel["unmask"][s])
+            for i in range(W.BLOCK):
+                if not sel["token_ambiguous"][s, i]:
+                    bad_tok += int(got["tokens"][s, i]) != int(sel["tokens"][s, i])
+        out.update(sequences_checked=dec, positions_checked=pos,
+                   decision_ambiguous=int(sel["decision_ambiguous"].sum()),
+                   token_ambiguous=int(sel["token_ambiguous"].sum()),
+                   decision_mismatches=bad_dec, token_mismatches=bad_tok,
+                   pmax_max_abs_err=pmax_err, pmax_outside_tol=bad_pmax)
+        ok &= bad_dec == 0 and bad_tok == 0 and bad_pmax == 0
+    out["pass"] = bool(ok)
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -482,6 +570,12 @@ def run_ours(args, cfg, tau, S, dist: Dist):
     torch.cuda.synchronize(dev)
     dist.barrier()
     t_wall1 = time.time()
+    # the timed step's outputs, for the parity block (compared after timing)
+    got = {"out": step.out.float().cpu().numpy() if step.attn else None}
+    if step.sel:
+        got.update(tokens=step.tokens.cpu().numpy(), unmask=step.unmask.cpu().numpy().view(np.uint32),
+                   pmax=step.pmax.cpu().numpy(), argmax=step.argmax.cpu().numpy(),
+                   masked=step.masked_host)
     # Per-call breakdown, outside the timed region: each call on its own
     # (one graph per call), L2 flushed before each step as above.
     n_bd = max(10, K // 4)
@@ -567,7 +661,8 @@ def run_ours(args, cfg, tau, S, dist: Dist):
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         if s_in is not None:
             s_in["n_scored"] = n_scored
-        line["cpu_baseline"] = cpu_baseline(cfg, a_in, s_in, tau, S, args.cpu_budget_s)
+        line["cpu_baseline"], line["parity"] = cpu_baseline(
+            cfg, a_in, s_in, tau, S, args.cpu_budget_s, None if step.active_only else got)
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
 

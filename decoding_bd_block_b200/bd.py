@@ -23,7 +23,7 @@ EXPORTED = ("bd_cache_commit", "bd_block_attn_workspace_size", "bd_block_attn",
             "bd_confidence_select_workspace_size", "bd_confidence_select",
             "bd_block_mask_attn", "bd_status_string", "bd_last_cuda_error_string",
             "bd_kernel_launches", "bd_confidence_select_noalloc", "bd_confidence_select_active",
-            "bd_masked_ce_workspace_size", "bd_masked_ce")
+            "bd_masked_ce_workspace_size", "bd_masked_ce", "bd_eval_exp2")
 BD_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 if not os.path.exists(_LIB_PATH):
@@ -74,6 +74,7 @@ _SIGS = {
                                     _P, _P, _P, ctypes.c_size_t, _P],
     "bd_masked_ce_workspace_size": [_I, _I, _I, _I, _I, _SZ],
     "bd_masked_ce": [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "bd_eval_exp2": [_P, _P, _P, _P, _I, _P],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -235,6 +236,13 @@ def bd_block_mask_attn(shape: bd_attn_shape, q, k, v, out, n_seqs, L, block, str
     _check("bd_block_mask_attn", _lib.bd_block_mask_attn(
         ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out), int(n_seqs), int(L),
         int(block), _stream(stream)))
+
+
+def bd_eval_exp2(x, y_poly, y_pair, y_mufu, stream=None):
+    """Diagnostic: the library's exponential approximations on the float32
+    tensor x (see include/bd.h)."""
+    _check("bd_eval_exp2", _lib.bd_eval_exp2(_ptr(x), _ptr(y_poly), _ptr(y_pair), _ptr(y_mufu),
+                                             int(x.numel()), _stream(stream)))
 
 
 def bd_kernel_launches() -> int:

@@ -255,12 +255,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     const uint32_t sbuf = tmem + lane_off + kColS + t * 128;
+    // A warp whose 32 rows are all padding of the last query tile (G * 32 not
+    // a multiple of 128) only keeps the barrier protocol: its P rows are never
+    // written, so P V gives garbage in output rows that are never stored.
+    const bool pad_warp = 32 * (r / 32) >= a.R;
     for (int j = 0; j < n_tiles && ok; ++j) {
       const int valid = min(kKeys, kBlock * (n_pg - 4 * j));
       // S_t(j) complete also means tile t's earlier products (P V of stage
       // j-1 included) have completed: none of tile t's MMAs is in flight.
       if (!tc::mbar_wait_warp(&s_full[t], j & 1, a.status)) { ok = false; break; }
       tc::tc_fence_after();
+      if (pad_warp) {
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&p_full[t]);
+        continue;
+      }
       uint32_t sr[128];
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc)

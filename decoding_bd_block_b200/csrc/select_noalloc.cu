@@ -14,7 +14,15 @@
 // process exits, whether or not this entry point is used.  Host code cannot
 // pass the variable's name to a kernel (on the host it names a stand-in, not
 // device memory), so its device address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, and cached.
+// cudaGetSymbolAddress, with that device current, and cached for the life of
+// the process (a cudaDeviceReset would leave the cached address stale).
+//
+// The scratch starts with the 16-byte header of the select workspace (the
+// row count, a status word, and the arrival and tile counters of the
+// single-kernel path), which the kernels expect to read as zero when a call
+// starts.  Every call clears it on the caller's stream before its kernels,
+// so a call that was cut short (or that overlapped another one) cannot
+// leave a later, properly ordered call reading stale counters.
 #include <mutex>
 
 #include <nvtx3/nvToolsExt.h>
@@ -68,6 +76,9 @@ static int noalloc_call(int32_t dtype, int32_t batch, int32_t hidden, int32_t vo
   cudaError_t e = cudaSuccess;
   void* scratch = bd::scratch_for_current_device(&e);
   if (!scratch) return bd::report_cuda_error(e);  // BD_ERR_CUDA, text kept for the caller
+  // the select kernels read the header as zero at the start of a call
+  e = cudaMemsetAsync(scratch, 0, 16, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return bd::report_cuda_error(e);
   return bd_confidence_select(dtype, batch, hidden, vocab, h, h_prev, w, masked_bits, tau,
                               sub_block, tokens, unmask_bits, pmax_out, argmax_out, scratch,
                               static_cast<size_t>(BD_NOALLOC_SCRATCH_BYTES), stream);

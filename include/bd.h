@@ -251,12 +251,16 @@ BD_API int bd_masked_ce(int32_t dtype, int32_t n_seqs, int32_t seq_len,
  * bf16 on a 148-SM B200 that is a batch above 24 at hidden 3584, above 48
  * at hidden 1536.  The call
  * allocates nothing.  Its first call on a device looks the array's device
- * address up (cudaGetSymbolAddress) with that device current; make that
- * first call before any stream capture on the device.  Every call on a
- * device shares the one array and leaves its contents behind for the next
- * (nothing in it has to start at zero: each call writes every part it
- * reads), so calls whose work overlaps on the GPU -- different streams, or
- * different host threads on one device -- race and must be serialised by the
+ * address up (cudaGetSymbolAddress) with that device current and keeps it
+ * for the life of the process: make that first call before any stream
+ * capture on the device, and do not use this call after a cudaDeviceReset.
+ * Every call on a device shares the one array.  Each call first clears the
+ * array's 16-byte header on `stream` (cudaMemsetAsync: the single-kernel
+ * path counts CTA arrivals and vocab tiles there and needs them zero at the
+ * start); the rest of the array holds the last call's packed rows and
+ * partials, which the next call overwrites before it reads them.  Calls
+ * whose work overlaps on the GPU -- different streams, or different host
+ * threads on one device -- race on the array and must be serialised by the
  * caller. */
 #define BD_NOALLOC_SCRATCH_BYTES (8u << 20)
 BD_API int bd_confidence_select_noalloc(int32_t dtype, int32_t batch, int32_t hidden,
@@ -282,6 +286,22 @@ BD_API int bd_confidence_select_noalloc(int32_t dtype, int32_t batch, int32_t hi
 BD_API int bd_block_mask_attn(const bd_attn_shape* shape, const void* q,
                        const void* k, const void* v, void* out,
                        int32_t n_seqs, int32_t L, int32_t block, void* stream);
+
+/* bd_eval_exp2 -- diagnostic: the library's exponential approximations.
+ *
+ * No counterpart in the method: the attention softmax and the LM-head
+ * statistics evaluate part of their exponentials 2^x with a polynomial on
+ * the FMA pipe (relative error below 2.7e-6 for -126 <= x <= 0) and the rest
+ * with the hardware approximation; this call evaluates them on given
+ * arguments so that a test can check those bounds on the device.
+ *   x       device, [n] float arguments
+ *   y_poly  device, [n] out: the scalar polynomial
+ *   y_pair  device, [n] out: the paired (two-lane) polynomial, on the pairs
+ *           (x[2i], x[2i+1])
+ *   y_mufu  device, [n] out: the hardware approximation (ex2.approx.ftz)
+ * BD_ERR_INVALID_ARG for a null pointer or n < 0. */
+BD_API int bd_eval_exp2(const float* x, float* y_poly, float* y_pair, float* y_mufu,
+                        int32_t n, void* stream);
 
 /* Human-readable name of a bd_status value. */
 BD_API const char* bd_status_string(int status);

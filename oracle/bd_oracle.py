@@ -456,7 +456,9 @@ def decode_loop(weights, prompt, n_blocks: int, tau: float, sub_block: int, *,
     ``[B]`` unmask words), ``ambiguous_at`` ((block, step) of the first
     decision flagged by reading R8, or None).  With ``trace``, also
     ``records``: per step (block, step, refresh flags ``[B]``, p_max of the
-    step, p_max of the exact step on the same tokens and cache).
+    step, p_max of the exact step on the same tokens and cache), ``h_prev``
+    (per decoded block, the ``[B, H]`` rows its position 0 was read from)
+    and ``cache`` (the :class:`OracleCache` after the loop).
     """
     E, Wq, Wk, Wv, Wo, W = (np.asarray(weights[n], np.float64)
                             for n in ("E", "Wq", "Wk", "Wv", "Wo", "W"))
@@ -484,10 +486,11 @@ def decode_loop(weights, prompt, n_blocks: int, tau: float, sub_block: int, *,
         h = hidden(x, q, k, v)
         commit(k, v)
         h_prev = h[:, BLOCK - 1]
-    toks, logs, records = [prompt], [], []
+    toks, logs, records, h_prev_in = [prompt], [], [], []
     steps = np.zeros((n_blocks, B), np.int64)
     ambiguous_at = None
     for b in range(n_blocks):
+        h_prev_in.append(h_prev.copy())
         tok = np.full((B, BLOCK), MASK_TOKEN, np.int64)
         log = []
         cached_sub = [None] * B  # active sub-block the DualCache was filled for
@@ -542,5 +545,5 @@ def decode_loop(weights, prompt, n_blocks: int, tau: float, sub_block: int, *,
     out = dict(tokens=np.concatenate(toks, 1), steps=steps, unmasked=logs,
                ambiguous_at=ambiguous_at)
     if trace:
-        out["records"] = records
+        out.update(records=records, h_prev=h_prev_in, cache=cache)
     return out

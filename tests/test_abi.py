@@ -61,3 +61,16 @@ def test_host_validation_without_gpu():
     d96 = bd.make_shape(12, 2, 96, "bf16")
     assert bd._lib.bd_block_mask_attn(ctypes.byref(d96), 1, 1, 1, 1, 1, 64, 32, None) == -2
     assert bd._lib.bd_block_mask_attn(ctypes.byref(shape), 1, 1, 1, 1, 1, 48, 32, None) == -1
+
+
+@pytest.mark.parametrize("hidden,vocab,fits,refused", [(3584, 152064, 24, 25), (1536, 151936, 48, 49)])
+def test_noalloc_size_limit_boundaries(hidden, vocab, fits, refused):
+    # bd_confidence_select_noalloc refuses a step whose scratch (the
+    # bd_confidence_select workspace) exceeds its fixed array: in bf16 on a
+    # 148-SM B200 the last accepted batch is 24 at hidden 3584 and 48 at
+    # hidden 1536 (the limits the header states).
+    from decoding_bd_block_b200 import bd
+    assert bd.bd_confidence_select_workspace_size("bf16", fits, hidden, vocab) \
+        <= bd.BD_NOALLOC_SCRATCH_BYTES
+    assert bd.bd_confidence_select_workspace_size("bf16", refused, hidden, vocab) \
+        > bd.BD_NOALLOC_SCRATCH_BYTES

@@ -120,15 +120,10 @@ def test_block_attn_longctx_sampled():
         assert err <= ATOL["bf16"], (s, err)
 
 
-def test_block_attn_growing_scores_rescale():
-    # Keys grow page by page (up to 4x), so the running max keeps rising across
-    # the KV stream and the online softmax must rescale its accumulator (about
-    # one rescale per query row).  Scores this large make the bf16 storage of
-    # the rotated q / K (the cache format) itself worth ~3e-2 against fp64, so
-    # the kernel is held to 2e-2 against the same computation with that
-    # storage rounding applied, and to that storage error + 2e-2 against the
-    # oracle.
-    from decoding_bd_block_b200.step import DecodeStep
+def _growing_case():
+    """Keys that grow page by page (up to 4x): the running max keeps rising
+    across the KV stream, so the online softmax must rescale its accumulator
+    (about one rescale per query row)."""
     cfg = dataclasses.replace(W.QWEN7B_RAGGED, name="bf16_growing", batch=2, prefix_range=(),
                               prefix_tokens=(3072, 1504), seed=103)
     a = W.make_attn_inputs(cfg)
@@ -137,16 +132,43 @@ def test_block_attn_growing_scores_rescale():
         ramp = (1.0 + np.arange(k.shape[0]) / 1024.0).astype(np.float32)[:, None, None]
         a["prefix_k"][s] = W.bf16_bits_from_f32(k * ramp)
     a["k_blk"] = W.bf16_bits_from_f32(W.f32_from_bf16_bits(a["k_blk"]) * 4.0)
+    return cfg, a
+
+
+def _run_growing():
+    from decoding_bd_block_b200.step import DecodeStep
+    cfg, a = _growing_case()
     step = DecodeStep(cfg, a, None)
     step.run_attn()
     torch.cuda.synchronize()
-    got = step.out.float().cpu().numpy()
+    return cfg, a, step.out.float().cpu().numpy()
+
+
+def test_block_attn_growing_scores_rescale():
+    # Reading: the bf16 path multiplies on the tensor cores, whose operands
+    # are bf16, so the rotated q and keys are rounded to bf16 before the
+    # products (whether the cache stores keys rotated or not).  Against the
+    # oracle with exactly that rounding applied the kernel stays within the
+    # bf16 bound; the error of the rounding itself against the fp64 oracle
+    # is reported (about 3.4e-2 on this input class, see the strict xfail
+    # below; about 2e-3 on the bf16 decoding workloads).
+    cfg, a, got = _run_growing()
     ref = oracle_block_attn(cfg, a)
     emu = bf16_storage_block_attn(cfg, a)
     for s in ref:
-        storage = float(np.abs(emu[s] - ref[s]).max())
-        assert float(np.abs(got[s] - emu[s]).max()) <= ATOL["bf16"]
-        assert float(np.abs(got[s] - ref[s]).max()) <= storage + ATOL["bf16"]
+        err_emu = float(np.abs(got[s] - emu[s]).max())
+        print(f"seq {s}: vs bf16-operand oracle {err_emu:.3e}, vs fp64 oracle "
+              f"{float(np.abs(got[s] - ref[s]).max()):.3e}, rounding alone "
+              f"{float(np.abs(emu[s] - ref[s]).max()):.3e}")
+        assert err_emu <= ATOL["bf16"]
+
+
+@pytest.mark.xfail(strict=True, reason="bf16 tensor-core operands: rounding the rotated q and keys "
+                   "alone is 3.4e-2 from the fp64 oracle on these growing keys (stated bound 2e-2)")
+def test_block_attn_growing_scores_vs_fp64_oracle():
+    cfg, a, got = _run_growing()
+    ref = oracle_block_attn(cfg, a)
+    assert max(float(np.abs(got[s] - ref[s]).max()) for s in ref) <= ATOL["bf16"]
 
 
 def test_block_attn_repeatable_and_after_commit():
@@ -347,3 +369,54 @@ def test_host_validation_errors_launch_nothing():
     with pytest.raises(bd.BdError) as e:
         bd.bd_block_attn(st.cache, q, q, q, torch.empty_like(q), ws, workspace_bytes=0)
     assert e.value.status == -4
+
+
+# ------------------------------------------- canary-padded output buffers
+CANARY, PAD = 0xA5, 4096
+
+
+def _canaried(shape, dtype):
+    """A tensor of `shape` inside a byte buffer with PAD canary bytes on each
+    side (16-byte alignment kept); returns (buffer, tensor)."""
+    n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+    buf = torch.full((n + 2 * PAD,), CANARY, dtype=torch.uint8, device="cuda")
+    return buf, buf[PAD:PAD + n].view(dtype).view(*shape)
+
+
+def _canaries_intact(buf):
+    return bool((buf[:PAD] == CANARY).all()) and bool((buf[-PAD:] == CANARY).all())
+
+
+@pytest.mark.parametrize("cfg", [W.TINY_F32, W.QWEN15B_STEP, ATTN_CASES[5]], ids=lambda c: c.name)
+def test_block_attn_writes_only_its_output(cfg):
+    # The output of bd_block_attn sits between canary bytes: after the call
+    # they are intact and the output equals that of the step's own buffer.
+    from decoding_bd_block_b200 import bd
+    _, _, step = _step(cfg, sel=False)
+    step.run_attn()
+    buf, out = _canaried(tuple(step.out.shape), step.out.dtype)
+    bd.bd_block_attn(step.cstate.cache, step.q, step.k_blk, step.v_blk, out, step.attn_ws)
+    torch.cuda.synchronize()
+    assert _canaries_intact(buf)
+    assert torch.equal(out, step.out)
+
+
+@pytest.mark.parametrize("cfg", [W.TINY_F32, W.QWEN15B_STEP, W.QWEN7B_RAGGED], ids=lambda c: c.name)
+def test_confidence_select_writes_only_its_outputs(cfg):
+    # tokens, unmask bits, p_max and argmax each sit between canary bytes.
+    from decoding_bd_block_b200 import bd
+    _, s, step = _step(cfg, attn=False)
+    step.run_select(0.9, 8)
+    torch.cuda.synchronize()
+    bt, tok = _canaried(tuple(step.tokens.shape), torch.int32)
+    bu, un = _canaried(tuple(step.unmask.shape), torch.int32)
+    bp, pm = _canaried(tuple(step.pmax.shape), torch.float32)
+    ba, am = _canaried(tuple(step.argmax.shape), torch.int32)
+    tok.copy_(step.tokens_in)
+    bd.bd_confidence_select(cfg.dtype, cfg.batch, cfg.hidden, cfg.vocab, step.h, step.h_prev,
+                            step.W, step.masked, 0.9, 8, tok, un, pm, am, step.sel_ws)
+    torch.cuda.synchronize()
+    assert all(_canaries_intact(b) for b in (bt, bu, bp, ba))
+    assert torch.equal(tok, step.tokens) and torch.equal(un, step.unmask)
+    assert torch.equal(am, step.argmax)
+    torch.testing.assert_close(torch.nan_to_num(pm), torch.nan_to_num(step.pmax), rtol=1e-5, atol=0)

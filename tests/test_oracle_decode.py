@@ -84,3 +84,64 @@ def test_exact_loop_tau1_one_token_per_step():
     for log in exact["unmasked"]:
         for u in log:
             assert all(bin(int(x)).count("1") == 1 for x in u)
+
+
+def _recompute(w, tokens):
+    """The single layer of reading R10 on whole sequences, without any cache:
+    per sequence x = E[tokens], q/k/v projections, the block-causal attention
+    recomputed over every token, h = x + attn Wo."""
+    E, Wq, Wk, Wv, Wo = (np.asarray(w[n], np.float64) for n in ("E", "Wq", "Wk", "Wv", "Wo"))
+    Hq, Hkv, d, th = KW["n_heads_q"], KW["n_heads_kv"], KW["head_dim"], KW["rope_theta"]
+    out = []
+    for s in range(tokens.shape[0]):
+        x = E[tokens[s]]
+        T = x.shape[0]
+        q = (x @ Wq).reshape(T, Hq, d)
+        k = (x @ Wk).reshape(T, Hkv, d)
+        v = (x @ Wv).reshape(T, Hkv, d)
+        att = O.full_sequence_attn(q, k, v, th)
+        out.append(dict(k=O.rope(k, np.arange(T), th), v=v, h=x + att.reshape(T, Hq * d) @ Wo))
+    return out
+
+
+@pytest.mark.parametrize("tau,dual", [(0.9, False), (0.3, False), (0.9, True)])
+def test_committed_blocks_and_h_prev_equal_a_full_recompute(tau, dual):
+    # [N1] key design 3: a decoded block's K/V become read-only context, as in
+    # an AR KV cache.  After the loop, every committed block must hold the
+    # rotated K and the V of its FINAL tokens at their absolute positions, and
+    # each block's position 0 must have been read from the last hidden row of
+    # the block before it, both as a cache-free recompute of the whole
+    # sequence under the block-causal mask gives them.  Committing the K/V of
+    # the last denoising step (one position still [MASK]) or taking h_prev
+    # from that step fails here.
+    w, p = weights(w_std=2.0), prompt(blocks=2)
+    n_blocks, S = 3, 8
+    r = O.decode_loop(w, p, n_blocks, tau, S, dual_cache=dual, trace=True, **KW)
+    assert not (r["tokens"] == O.MASK_TOKEN).any()
+    ref = _recompute(w, r["tokens"])
+    T = r["tokens"].shape[1]
+    for s, rs in enumerate(ref):
+        np.testing.assert_allclose(r["cache"].k[s], rs["k"], rtol=0, atol=1e-10)
+        np.testing.assert_allclose(r["cache"].v[s], rs["v"], rtol=0, atol=1e-12)
+        assert r["cache"].length(s) == T
+    n_prompt = p.shape[1] // 32
+    for b in range(n_blocks):
+        want = np.stack([rs["h"][32 * (n_prompt + b) - 1] for rs in ref])
+        np.testing.assert_allclose(r["h_prev"][b], want, rtol=0, atol=1e-10)
+
+
+def test_committed_pin_catches_a_stale_commit(monkeypatch):
+    # The pin above must fail on a plausible slip: here the oracle's commit is
+    # fed the K/V of the block with one position still [MASK] (as if the last
+    # denoising step's projections were committed).
+    w, p = weights(w_std=2.0), prompt()
+    real_commit = O.OracleCache.commit
+    def stale_commit(self, s, k_new, v_new):
+        k_new = np.array(k_new, np.float64)
+        if self.length(s) >= 32:            # a decoded block, not the prompt
+            k_new[-1] += 1.0                # its last position's K changed
+        return real_commit(self, s, k_new, v_new)
+    monkeypatch.setattr(O.OracleCache, "commit", stale_commit)
+    r = O.decode_loop(w, p, 2, 0.9, 8, trace=True, **KW)
+    ref = _recompute(w, r["tokens"])
+    assert not np.allclose(r["cache"].k[0], ref[0]["k"], atol=1e-10)
