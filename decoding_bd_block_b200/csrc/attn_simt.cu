@@ -243,54 +243,55 @@ __global__ void __launch_bounds__(256) attn_split_simt_kernel(
   }
 }
 
-// grid (32, Hq, batch), D threads: merge the chunks of one output row.  The
-// chunks' (m, l, O) are read eight at a time, all loads in flight, and
-// folded into a running (max, sum, acc) in base-2 exponent units.
+// grid (Hq, batch), 256 threads: merge the chunks of one query head's 32
+// output rows.  Thread i owns row i / 8 and the D / 8 consecutive elements
+// (i % 8) * D / 8 ..; the eight threads of a row read its partial O rows as
+// contiguous 16-byte vectors.  Two passes over the chunks: the largest m
+// (base-2 exponent units), then the weighted sums of l and O.
 template <typename T, int D>
-__global__ void __launch_bounds__(D) attn_merge_kernel(const int32_t* __restrict__ n_blocks,
-                                                       const float* __restrict__ part_o,
-                                                       const float* __restrict__ part_ml,
-                                                       T* __restrict__ out, int Hq, int ppc,
-                                                       int max_chunks) {
-  const int t = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+__global__ void __launch_bounds__(256) attn_merge_kernel(const int32_t* __restrict__ n_blocks,
+                                                         const float* __restrict__ part_o,
+                                                         const float* __restrict__ part_ml,
+                                                         T* __restrict__ out, int Hq, int ppc,
+                                                         int max_chunks) {
+  constexpr int E = D / 8;  // elements per thread
+  const int h = blockIdx.x, s = blockIdx.y;
+  const int t = threadIdx.x / 8, d0 = (threadIdx.x % 8) * E;
   griddep_wait();  // the split kernel's partials
   griddep_launch_dependents();
   const int total = max(n_blocks[s], 0) + 1;
   if (total <= ppc) return;  // written directly by the split kernel
   const int nch = min((total + ppc - 1) / ppc, max_chunks);
   const size_t base = (static_cast<size_t>(s) * Hq + h) * max_chunks;
-  float M = -INFINITY, L = 0.f, acc = 0.f;
-  for (int c0 = 0; c0 < nch; c0 += 8) {
-    float m[8], l[8], o[8];
+  const float2* ml = reinterpret_cast<const float2*>(part_ml);
+  float M = -INFINITY;
+  for (int c = 0; c < nch; ++c) M = fmaxf(M, ml[(base + c) * kBlock + t].x);
+  float L = 0.f, acc[E];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int c = c0 + u;
-      m[u] = -INFINITY;
-      l[u] = 0.f;
-      o[u] = 0.f;
-      if (c < nch) {
-        const size_t r = (base + c) * kBlock + t;
-        const float2 ml = reinterpret_cast<const float2*>(part_ml)[r];
-        m[u] = ml.x;
-        l[u] = ml.y;
-        o[u] = part_o[r * D + threadIdx.x];
-      }
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll 2
+  for (int c = 0; c < nch; ++c) {
+    const size_t r = (base + c) * kBlock + t;
+    const float2 v = ml[r];
+    const float w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
+    L = fmaf(v.y, w, L);
+    const float4* o = reinterpret_cast<const float4*>(part_o + r * D + d0);
+#pragma unroll
+    for (int e = 0; e < E / 4; ++e) {
+      const float4 x = o[e];
+      acc[4 * e + 0] = fmaf(x.x, w, acc[4 * e + 0]);
+      acc[4 * e + 1] = fmaf(x.y, w, acc[4 * e + 1]);
+      acc[4 * e + 2] = fmaf(x.z, w, acc[4 * e + 2]);
+      acc[4 * e + 3] = fmaf(x.w, w, acc[4 * e + 3]);
     }
-    float Mn = M;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) Mn = fmaxf(Mn, m[u]);
-    const float sc = M == -INFINITY ? 0.f : exp2f(M - Mn);
-    L *= sc;
-    acc *= sc;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float w = m[u] == -INFINITY ? 0.f : exp2f(m[u] - Mn);
-      L += l[u] * w;
-      acc += o[u] * w;
-    }
-    M = Mn;
   }
-  out[((static_cast<size_t>(s) * kBlock + t) * Hq + h) * D + threadIdx.x] = from_f32<T>(acc / L);
+  const float inv = 1.f / L;
+  T res[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) res[e] = from_f32<T>(acc[e] * inv);
+  uint4* dst = reinterpret_cast<uint4*>(out + ((static_cast<size_t>(s) * kBlock + t) * Hq + h) * D + d0);
+#pragma unroll
+  for (int e = 0; e < static_cast<int>(E * sizeof(T) / 16); ++e) dst[e] = reinterpret_cast<const uint4*>(res)[e];
 }
 
 // -------------------------------------------------------------- host side
@@ -382,7 +383,7 @@ static cudaError_t launch_attn_t(const bd_attn_shape& sh, const bd_kv_cache& c, 
                        reinterpret_cast<int32_t*>(w + p.off_status), st);
     if (e != cudaSuccess) return e;
     if (p.max_chunks > 1) {
-      e = launch_pdl(attn_merge_kernel<T, D>, dim3(kBlock, sh.n_heads_q, c.batch), dim3(D), 0, st,
+      e = launch_pdl(attn_merge_kernel<T, D>, dim3(sh.n_heads_q, c.batch), dim3(256), 0, st,
                      c.n_blocks, part_o, part_ml, static_cast<T*>(out), sh.n_heads_q,
                      p.pages_per_chunk, p.max_chunks);
       if (e != cudaSuccess) return e;
@@ -398,7 +399,7 @@ static cudaError_t launch_attn_t(const bd_attn_shape& sh, const bd_kv_cache& c, 
       ws_blk, part_o, part_ml, static_cast<T*>(out), sh.n_heads_q, sh.n_heads_kv,
       p.pages_per_chunk, p.max_chunks);
   if (p.max_chunks > 1)
-    attn_merge_kernel<T, D><<<dim3(kBlock, sh.n_heads_q, c.batch), D, 0, st>>>(
+    attn_merge_kernel<T, D><<<dim3(sh.n_heads_q, c.batch), 256, 0, st>>>(
         c.n_blocks, part_o, part_ml, static_cast<T*>(out), sh.n_heads_q, p.pages_per_chunk,
         p.max_chunks);
   count_launches(p.max_chunks > 1 ? 2 : 1);

@@ -283,7 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int k = 0; k < 128; ++k) mk[k & 3] = fmaxf(mk[k & 3], __uint_as_float(sr[k]));
+      for (int k = 0; k < 128; k += 2)
+        mk[(k >> 1) & 3] = tc::fmax3(mk[(k >> 1) & 3], __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
       const float mt = fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])) * scale;
       const float m_new = fmaxf(m, mt);
       const bool rescale = (m == -INFINITY) || (m_new - m > kRescaleThreshold);

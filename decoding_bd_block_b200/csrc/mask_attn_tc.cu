@@ -232,15 +232,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int cc = 0; cc < 4; ++cc)
         tc::tmem_ld_32x32b_x32(sbuf + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
       tc::tmem_ld_wait();
+      // Visible 32-key chunks of this key tile for this warp's rows (4 bits,
+      // warp-uniform).  When D is a multiple of 32 a warp's 32 rows lie in
+      // one block and so does each 32-key chunk, so a chunk is wholly
+      // visible or wholly masked: masked chunks get no exponentials and P = 0.
+      // Otherwise partly visible tiles are masked element by element.
+      uint32_t cmask = 0xFu;
       if (kv_kind[j] != 2) {  // warp-uniform: partly visible key tile
         const int j0 = kv_list[j] * kT;
+        if (a.D % 32 == 0) {
+          const int iw = qt * kT + 32 * q;  // the warp's first row
+          cmask = 0u;
 #pragma unroll
-        for (int k = 0; k < 128; ++k)
-          if (!pair_visible(i, j0 + k, a.L, a.D)) sr[k] = __float_as_uint(-INFINITY);
+          for (int c = 0; c < 4; ++c) cmask |= pair_visible(iw, j0 + 32 * c, a.L, a.D) ? 1u << c : 0u;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 128; ++k)
+            if (!pair_visible(i, j0 + k, a.L, a.D)) sr[k] = __float_as_uint(-INFINITY);
+        }
       }
       float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int k = 0; k < 128; ++k) mk[k & 3] = fmaxf(mk[k & 3], __uint_as_float(sr[k]));
+      for (int c = 0; c < 4; ++c)
+        if ((cmask >> c) & 1u) {
+#pragma unroll
+          for (int k = 32 * c; k < 32 * c + 32; k += 2)
+            mk[(k >> 1) & 3] = tc::fmax3(mk[(k >> 1) & 3], __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
+        }
       const float mt = fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])) * scale;
       const float m_new = fmaxf(m, mt);
       // a row with no visible key in this tile keeps m = -inf until one shows up
@@ -254,22 +272,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(neg_m, neg_m);
       float2 rk[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {  // packs in place: sr[k] <- (p_2k, p_2k+1)
-        // paired fp32 arithmetic; a quarter of the pairs' exponentials on the
-        // FMA pipe, the rest on MUFU (which gives exact zeros for masked,
-        // -inf, scores; poly_exp2x2 floors at 2^-126, so those are zeroed)
-        const float s0 = __uint_as_float(sr[2 * k]), s1 = __uint_as_float(sr[2 * k + 1]);
-        const float2 x = ffma2(make_float2(s0, s1), sc2, nm2);
-        float2 e;
-        if ((k & 3) == 3) {
-          e = poly_exp2x2(x);
-          e.x = s0 == -INFINITY ? 0.f : e.x;
-          e.y = s1 == -INFINITY ? 0.f : e.y;
+      for (int c = 0; c < 4; ++c) {
+        if ((cmask >> c) & 1u) {
+#pragma unroll
+          for (int k = 16 * c; k < 16 * c + 16; ++k) {  // packs in place: sr[k] <- (p_2k, p_2k+1)
+            // paired fp32 arithmetic; a quarter of the pairs' exponentials on
+            // the FMA pipe, the rest on MUFU (which gives exact zeros for
+            // masked, -inf, scores; poly_exp2x2 floors at 2^-126, so those
+            // are zeroed)
+            const float s0 = __uint_as_float(sr[2 * k]), s1 = __uint_as_float(sr[2 * k + 1]);
+            const float2 x = ffma2(make_float2(s0, s1), sc2, nm2);
+            float2 e;
+            if ((k & 3) == 3) {
+              e = poly_exp2x2(x);
+              e.x = s0 == -INFINITY ? 0.f : e.x;
+              e.y = s1 == -INFINITY ? 0.f : e.y;
+            } else {
+              e = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            }
+            rk[k & 1] = fadd2(rk[k & 1], e);
+            sr[k] = tc::pack_bf16x2(e.x, e.y);
+          }
         } else {
-          e = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+#pragma unroll
+          for (int k = 16 * c; k < 16 * c + 16; ++k) sr[k] = 0u;
         }
-        rk[k & 1] = fadd2(rk[k & 1], e);
-        sr[k] = tc::pack_bf16x2(e.x, e.y);
       }
       l = l * alpha + ((rk[0].x + rk[0].y) + (rk[1].x + rk[1].y));
       const bool need = rescale && j > 0;

@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(1024) gather_rows_kernel(
     const int nvec = H * static_cast<int>(sizeof(T)) / 16;  // H * sizeof(T) % 16 == 0
     const uint4* s4 = reinterpret_cast<const uint4*>(src);
     uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll 4
     for (int x = lane; x < nvec; x += 32) d4[x] = s4[x];
   }
   if (s == B - 1) {
@@ -162,21 +163,49 @@ __global__ void __launch_bounds__(1024) merge_select_kernel(
   }
   const int parts = grouped ? n_split / ((count[0] + 255) / 256) : n_split;
   {
+    // Two passes over the row's partials, all of a lane's loads in flight:
+    // the largest max, then sum exp and the lowest argmax attaining it.
+    constexpr int kPer = 8;  // partials per lane kept in registers (parts <= 256)
     const int i = warp;
-    Stat st = stat_empty();
+    float s_sum = 0.f;
+    int a_min = 0x7fffffff;
+    float M = -INFINITY;
     if ((bits >> i) & 1u) {
       const size_t base = static_cast<size_t>(posrow[s * kBlock + i]) * n_split;
-      for (int k = lane; k < parts; k += 32) st = stat_combine(st, Stat{pm[base + k], ps[base + k], pa[base + k]});
+      float m[kPer], sv[kPer];
+      int av[kPer];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const Stat other{__shfl_xor_sync(0xffffffffu, st.m, o), __shfl_xor_sync(0xffffffffu, st.s, o),
-                         __shfl_xor_sync(0xffffffffu, st.a, o)};
-        st = stat_combine(st, other);
+      for (int u = 0; u < kPer; ++u) {
+        const int k = lane + 32 * u;
+        const bool in = k < parts;
+        m[u] = in ? pm[base + k] : -INFINITY;
+        sv[u] = in ? ps[base + k] : 0.f;
+        av[u] = in ? pa[base + k] : 0x7fffffff;
       }
+      for (int k = lane + 32 * kPer; k < parts; k += 32) {  // more than 256 partials
+        const Stat x = stat_combine(Stat{m[0], sv[0], av[0]}, Stat{pm[base + k], ps[base + k], pa[base + k]});
+        m[0] = x.m;
+        sv[0] = x.s;
+        av[0] = x.a;
+      }
+      float lm = m[0];
+#pragma unroll
+      for (int u = 1; u < kPer; ++u) lm = fmaxf(lm, m[u]);
+      M = warp_max(lm);
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+          if (m[u] != -INFINITY) s_sum += sv[u] * exp2f((m[u] - M) * kLog2e);
+          if (m[u] == M) a_min = min(a_min, av[u]);
+        }
+      }
+      s_sum = warp_sum(s_sum);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a_min = min(a_min, __shfl_xor_sync(0xffffffffu, a_min, o));
     }
     if (lane == 0) {
-      sp[i] = st.s > 0.f ? 1.f / st.s : 0.f;
-      stok[i] = st.a;
+      sp[i] = s_sum > 0.f ? 1.f / s_sum : 0.f;
+      stok[i] = a_min;
     }
   }
   __syncthreads();

@@ -77,11 +77,6 @@ struct SelectTcArgs {
   int32_t* status;
 };
 
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
 
 // Folds 32 logits of one row -- vocab entries vbase .. vbase + 31, the first
 // n of them valid (kFull: all 32) -- into the thread's running statistics.
@@ -95,14 +90,14 @@ __device__ __forceinline__ void fold_row32(const uint32_t (&r)[32], int n, int v
   for (int i = 0; i < 32; ++i) x[i] = (kFull || i < n) ? __uint_as_float(r[i]) : -INFINITY;
   float mk[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) mk[k] = fmax3(x[8 * k], x[8 * k + 1], x[8 * k + 2]);
+  for (int k = 0; k < 4; ++k) mk[k] = tc::fmax3(x[8 * k], x[8 * k + 1], x[8 * k + 2]);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) mk[k] = fmax3(mk[k], x[8 * k + 3], x[8 * k + 4]);
+  for (int k = 0; k < 4; ++k) mk[k] = tc::fmax3(mk[k], x[8 * k + 3], x[8 * k + 4]);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) mk[k] = fmax3(mk[k], x[8 * k + 5], x[8 * k + 6]);
+  for (int k = 0; k < 4; ++k) mk[k] = tc::fmax3(mk[k], x[8 * k + 5], x[8 * k + 6]);
 #pragma unroll
   for (int k = 0; k < 4; ++k) mk[k] = fmaxf(mk[k], x[8 * k + 7]);
-  const float mx = fmaxf(fmax3(mk[0], mk[1], mk[2]), mk[3]);
+  const float mx = fmaxf(tc::fmax3(mk[0], mk[1], mk[2]), mk[3]);
   if (mx == -INFINITY) return;
   const float m_new = fmaxf(run.m, mx);
   if (mx > run.m) {  // a new running maximum: its lowest index in the chunk
