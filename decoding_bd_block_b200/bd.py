@@ -23,7 +23,8 @@ EXPORTED = ("bd_cache_commit", "bd_block_attn_workspace_size", "bd_block_attn",
             "bd_confidence_select_workspace_size", "bd_confidence_select",
             "bd_block_mask_attn", "bd_status_string", "bd_last_cuda_error_string",
             "bd_kernel_launches", "bd_confidence_select_noalloc", "bd_confidence_select_active",
-            "bd_masked_ce_workspace_size", "bd_masked_ce", "bd_eval_exp2")
+            "bd_masked_ce_workspace_size", "bd_masked_ce", "bd_eval_exp2",
+            "bd_device_check_status")
 BD_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 if not os.path.exists(_LIB_PATH):
@@ -75,6 +76,7 @@ _SIGS = {
     "bd_masked_ce_workspace_size": [_I, _I, _I, _I, _I, _SZ],
     "bd_masked_ce": [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "bd_eval_exp2": [_P, _P, _P, _P, _I, _P],
+    "bd_device_check_status": [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32), _I],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -247,6 +249,30 @@ def bd_eval_exp2(x, y_poly, y_pair, y_mufu, stream=None):
 
 def bd_kernel_launches() -> int:
     return int(_lib.bd_kernel_launches())
+
+
+def device_check_status(lib=None, reset: bool = True):
+    """(code, detail) of the device-side index checks of ``lib`` (default:
+    this library, which has none and raises BD_ERR_UNSUPPORTED); see
+    include/bd.h."""
+    lib = _lib if lib is None else lib
+    code, detail = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check("bd_device_check_status", lib.bd_device_check_status(
+        ctypes.byref(code), ctypes.byref(detail), 1 if reset else 0))
+    return int(code.value), int(detail.value)
+
+
+_CHECKS_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbd_checks.so")
+
+
+def checks_library():
+    """The same library built with the device-side index checks
+    (libbd_checks.so): a ctypes handle whose entry points take the same
+    arguments as this module's (marshal them with the helpers here)."""
+    lib = ctypes.CDLL(_CHECKS_PATH)
+    for name, args in _SIGS.items():
+        getattr(lib, name).argtypes = args
+    return lib
 
 
 def raw_call(name, *args):

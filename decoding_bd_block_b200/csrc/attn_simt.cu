@@ -209,6 +209,7 @@ __global__ void __launch_bounds__(256) attn_split_simt_kernel(
     const T* vp;
     if (p < nb) {
       const int page = page_table[static_cast<size_t>(s) * max_blocks + p];
+      if (threadIdx.x == 0) BD_CHECK(page >= 0 && page < n_pages, kCheckPageId, page);
       if (page < 0 || page >= n_pages) continue;  // CTA-uniform; host-validated
       kp = pages + ((static_cast<size_t>(page) * 2 + 0) * Hkv + g) * kBlock * D;
       vp = pages + ((static_cast<size_t>(page) * 2 + 1) * Hkv + g) * kBlock * D;
@@ -516,3 +517,9 @@ cudaError_t launch_block_mask_attn(const bd_attn_shape& sh, const void* q, const
 }
 
 }  // namespace bd
+
+#ifdef BD_DEVICE_CHECKS
+namespace bd {
+cudaError_t check_word_attn_simt(int* host2, bool reset) { return read_check_word(host2, reset); }
+}  // namespace bd
+#endif

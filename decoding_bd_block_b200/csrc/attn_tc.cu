@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pg = -1;  // -1: the current block's page in the workspace
     if (p < nb) {
       pg = a.page_table[static_cast<size_t>(s) * a.max_blocks + p];
+      BD_CHECK(pg >= 0 && pg < a.n_pages, kCheckPageId, pg);
       if (pg < 0 || pg >= a.n_pages) pg = -2;  // host-validated; read zeros if not
     }
     pages[i] = pg;
@@ -203,18 +204,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t id_qk = tc::idesc_bf16_f32(128, kKeys);
       const uint32_t id_pv = tc::idesc_bf16_f32_bmn(128, kD);
-      auto slot_addr = [&](int b) { return sbase + kOffKV + (b % kSlots) * kKVBytes; };
       auto full = [&](int b) { return tc::mbar_wait(&kv_full[b % kSlots], (b / kSlots) & 1, a.status); };
+      // Shared-memory descriptors built once; a stage, a query tile or a
+      // K-step only moves the start-address field (bits [0,14), 16-byte
+      // units), so each MMA costs two 64-bit adds.  The issuing thread shares
+      // its SM sub-partition with softmax warps, so every instruction it
+      // saves keeps the tensor core fed.
+      const uint64_t qdesc0 = tc::sdesc_kmajor_sw128(sbase + kOffQ);
+      const uint64_t kdesc0 = tc::sdesc_kmajor_sw128(sbase + kOffKV);
+      const uint64_t vdesc0 = tc::sdesc_mnmajor_sw128(sbase + kOffKV, kKVBytes / 2);
+      constexpr uint64_t kSlotStep = kKVBytes >> 4, kQStep = kQTileBytes >> 4;
+      constexpr uint64_t kHalfStep = (kKVBytes / 2) >> 4;  // the second 64 of d (Q and K alike)
+      static_assert(kQTileBytes / 2 == kKVBytes / 2, "Q and K tiles split d at the same offset");
       auto issue_qk = [&](int t, int j) {  // S_t = Q_t K_j^T, K = d: 8 steps of 16
-        const uint32_t qaddr = sbase + kOffQ + t * kQTileBytes;
-        const uint32_t kaddr = slot_addr(2 * j);
+        const uint64_t qd = qdesc0 + static_cast<uint64_t>(t) * kQStep;
+        const uint64_t kd = kdesc0 + static_cast<uint64_t>((2 * j) % kSlots) * kSlotStep;
+        const uint32_t d = tmem + kColS + t * 128;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32;
-          tc::mma_bf16_ss(tmem + kColS + t * 128,
-                          tc::sdesc_kmajor_sw128(qaddr + (kk >> 2) * (kQTileBytes / 2) + off),
-                          tc::sdesc_kmajor_sw128(kaddr + (kk >> 2) * (kKVBytes / 2) + off), id_qk,
-                          kk != 0);
+          const uint64_t o = (kk >> 2) * kHalfStep + (kk & 3) * 2;  // + 32 bytes per K-step
+          tc::mma_bf16_ss(d, qd + o, kd + o, id_qk, kk != 0);
         }
         tc::mma_commit(&s_full[t]);
       };
@@ -224,16 +233,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) tc::mma_commit(&kv_empty[0]);  // K_0 has been read once its products are done
       for (int j = 0; j < n_tiles && ok; ++j) {
         const bool more = j + 1 < n_tiles;
-        const uint32_t vaddr = slot_addr(2 * j + 1);
+        const uint64_t vd = vdesc0 + static_cast<uint64_t>((2 * j + 1) % kSlots) * kSlotStep;
         for (int t = 0; t < nq && ok; ++t) {
           if (!tc::mbar_wait(&p_full[t], j & 1, a.status)) { ok = false; break; }
           if (t == 0 && !full(2 * j + 1)) { ok = false; break; }
           tc::tc_fence_after();
+          const uint32_t dO = tmem + kColO + t * 128, aP = tmem + kColS + t * 128;
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk)  // O_t += P_t V_j, K = keys: 8 steps of 16
-            tc::mma_bf16_ts(tmem + kColO + t * 128, tmem + kColS + t * 128 + kk * 8,
-                            tc::sdesc_mnmajor_sw128(vaddr + kk * 16 * 128, kKVBytes / 2), id_pv,
-                            (j | kk) != 0);
+            tc::mma_bf16_ts(dO, aP + kk * 8, vd + kk * ((16 * 128) >> 4), id_pv, (j | kk) != 0);
           tc::mma_commit(&pv_done[t]);
           if (t == nq - 1) tc::mma_commit(&kv_empty[(2 * j + 1) % kSlots]);  // V_j read
           if (more) {
@@ -525,3 +533,9 @@ cudaError_t launch_attn_tc(const bd_attn_shape& sh, const bd_kv_cache& c, int pp
 }
 
 }  // namespace bd
+
+#ifdef BD_DEVICE_CHECKS
+namespace bd {
+cudaError_t check_word_attn_tc(int* host2, bool reset) { return read_check_word(host2, reset); }
+}  // namespace bd
+#endif

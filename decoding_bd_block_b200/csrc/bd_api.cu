@@ -91,6 +91,32 @@ const char* bd_last_cuda_error_string(void) { return g_cuda_err; }
 
 long long bd_kernel_launches(void) { return bd::g_launches.load(std::memory_order_relaxed); }
 
+int bd_device_check_status(int32_t* code, int32_t* detail, int32_t reset) {
+#ifdef BD_DEVICE_CHECKS
+  if (!code || !detail) return BD_ERR_INVALID_ARG;
+  *code = 0;
+  *detail = 0;
+  cudaError_t (*const units[])(int*, bool) = {bd::check_word_commit, bd::check_word_attn_tc,
+                                              bd::check_word_attn_simt, bd::check_word_select,
+                                              bd::check_word_ce};
+  for (auto unit : units) {
+    int w[2] = {0, 0};
+    const int st = cuda_status(unit(w, reset != 0));
+    if (st) return st;
+    if (*code == 0 && w[0] != 0) {
+      *code = w[0];
+      *detail = w[1];
+    }
+  }
+  return BD_OK;
+#else
+  (void)code;
+  (void)detail;
+  (void)reset;
+  return BD_ERR_UNSUPPORTED;
+#endif
+}
+
 int bd_cache_commit(const bd_attn_shape* sh, bd_kv_cache* c, const void* k, const void* v,
                     const int32_t* seq_ids, int32_t n_seqs, int32_t n_new_blocks, void* stream) {
   NvtxRange nvtx_range("bd_cache_commit");

@@ -224,6 +224,46 @@ __device__ __forceinline__ void no_decision_sequence(int s, uint32_t* unmask, fl
   if (argmax_out) argmax_out[s * kBlock + i] = -2;
 }
 
+// ------------------------------------------------------ device-side checks
+// Built with -DBD_DEVICE_CHECKS (the library variant libbd_checks.so), kernels
+// check the indices they read from device memory (page ids, packed-row
+// indices, target ids) before using them.  A failed check is handled as in
+// the normal build (the access is skipped: zeros are read, nothing is
+// written) and is also recorded in a status word {code, detail}, the first
+// failure winning; bd_device_check_status() reports and clears it.  No trap,
+// no fault: the kernel runs to completion.  Without the flag the checks
+// compile to nothing.
+enum : int { kCheckNone = 0, kCheckPageId = 1, kCheckRowIndex = 2, kCheckTargetId = 3 };
+#ifdef BD_DEVICE_CHECKS
+// one word per translation unit (internal linkage; read by check_word_<unit>)
+static __device__ int g_check_word[2];
+__device__ __forceinline__ void check_fail(int code, int detail) {
+  if (atomicCAS(&g_check_word[0], 0, code) == 0) g_check_word[1] = detail;
+}
+#define BD_CHECK(ok, code, detail)        \
+  do {                                    \
+    if (!(ok)) ::bd::check_fail(code, detail); \
+  } while (0)
+static inline cudaError_t read_check_word(int* host2, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(host2, g_check_word, sizeof(g_check_word));
+  if (e == cudaSuccess && reset) {
+    const int zero[2] = {0, 0};
+    e = cudaMemcpyToSymbol(g_check_word, zero, sizeof(zero));
+  }
+  return e;
+}
+#else
+#define BD_CHECK(ok, code, detail) \
+  do {                             \
+  } while (0)
+#endif
+// The check words of the units that check (defined only with the flag).
+cudaError_t check_word_commit(int* host2, bool reset);
+cudaError_t check_word_attn_tc(int* host2, bool reset);
+cudaError_t check_word_attn_simt(int* host2, bool reset);
+cudaError_t check_word_select(int* host2, bool reset);
+cudaError_t check_word_ce(int* host2, bool reset);
+
 // Process-wide count of kernels enqueued by the library (bd_kernel_launches).
 void count_launches(int n);
 // Records a CUDA error for bd_last_cuda_error_string(); returns BD_ERR_CUDA

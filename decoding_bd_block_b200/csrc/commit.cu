@@ -27,6 +27,7 @@ __global__ void __launch_bounds__(128) cache_commit_kernel(
 
   if (t == 0 && threadIdx.x == 0) n_blocks[s] = first + a.n_new_blocks;
   const int page = page_table[static_cast<size_t>(s) * max_blocks + first + t / kBlock];
+  BD_CHECK(page >= 0 && page < n_pages, kCheckPageId, page);
   if (page < 0 || page >= n_pages) return;  // host-validated; never write outside the pool
   const int row = t % kBlock;
   const size_t span = static_cast<size_t>(kBlock) * a.n_new_blocks;
@@ -66,3 +67,9 @@ cudaError_t launch_cache_commit(const bd_attn_shape& sh, const bd_kv_cache& c, c
 }
 
 }  // namespace bd
+
+#ifdef BD_DEVICE_CHECKS
+namespace bd {
+cudaError_t check_word_commit(int* host2, bool reset) { return read_check_word(host2, reset); }
+}  // namespace bd
+#endif

@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(256) ce_merge_kernel(
     st = stat_combine(st, other);
   }
   const int y = tgt[r];
+  if (lane == 0) BD_CHECK(y >= 0 && y < V, kCheckTargetId, y);
   float dot = 0.f;
   if (y >= 0 && y < V) {
     const T* wr = w + static_cast<size_t>(y) * H;
@@ -267,3 +268,9 @@ cudaError_t launch_masked_ce(int dtype, int n_seqs, int seq_len, int hidden, int
 }
 
 }  // namespace bd
+
+#ifdef BD_DEVICE_CHECKS
+namespace bd {
+cudaError_t check_word_ce(int* host2, bool reset) { return read_check_word(host2, reset); }
+}  // namespace bd
+#endif

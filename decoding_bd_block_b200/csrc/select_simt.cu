@@ -51,8 +51,16 @@ __global__ void __launch_bounds__(1024) gather_rows_kernel(
     const int nvec = H * static_cast<int>(sizeof(T)) / 16;  // H * sizeof(T) % 16 == 0
     const uint4* s4 = reinterpret_cast<const uint4*>(src);
     uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll 4
-    for (int x = lane; x < nvec; x += 32) d4[x] = s4[x];
+    // eight 16-byte loads in flight per lane before their stores
+    for (int x0 = lane; x0 < nvec; x0 += 32 * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (x0 + 32 * u < nvec) v[u] = s4[x0 + 32 * u];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (x0 + 32 * u < nvec) d4[x0 + 32 * u] = v[u];
+    }
   }
   if (s == B - 1) {
     const int total = off + __popc(bits);
@@ -171,7 +179,10 @@ __global__ void __launch_bounds__(1024) merge_select_kernel(
     int a_min = 0x7fffffff;
     float M = -INFINITY;
     if ((bits >> i) & 1u) {
-      const size_t base = static_cast<size_t>(posrow[s * kBlock + i]) * n_split;
+      int prow = posrow[s * kBlock + i];
+      if (lane == 0) BD_CHECK(prow >= 0 && prow < count[0], kCheckRowIndex, prow);
+      prow = (prow >= 0 && prow < count[0]) ? prow : 0;  // written by the gather kernel
+      const size_t base = static_cast<size_t>(prow) * n_split;
       float m[kPer], sv[kPer];
       int av[kPer];
 #pragma unroll
@@ -335,3 +346,9 @@ cudaError_t launch_confidence_select(int dtype, int batch, int hidden, int vocab
 }
 
 }  // namespace bd
+
+#ifdef BD_DEVICE_CHECKS
+namespace bd {
+cudaError_t check_word_select(int* host2, bool reset) { return read_check_word(host2, reset); }
+}  // namespace bd
+#endif

@@ -303,6 +303,23 @@ BD_API int bd_block_mask_attn(const bd_attn_shape* shape, const void* q,
 BD_API int bd_eval_exp2(const float* x, float* y_poly, float* y_pair, float* y_mufu,
                         int32_t n, void* stream);
 
+/* bd_device_check_status -- diagnostic: the device-side index checks.
+ *
+ * No counterpart in the method.  The library built with BD_DEVICE_CHECKS
+ * defined (libbd_checks.so; `python -m decoding_bd_block_b200.build`
+ * builds it beside libbd.so) checks, inside its kernels, the indices it reads
+ * from device memory: cache page ids (commit, block attention), packed-row
+ * indices (confidence select) and target ids (masked CE).  A failed check
+ * skips the access as the normal build does (zeros are read, nothing is
+ * written) and records {code, detail}: the first failure since the last
+ * reset wins.  This call copies that record to the host (it waits for the
+ * device), and clears it when `reset` is nonzero.
+ *   code    host, out: 0 none, 1 page id outside [0, n_pages), 2 packed-row
+ *           index out of range, 3 target id outside [0, vocab)
+ *   detail  host, out: the offending value
+ * Returns BD_ERR_UNSUPPORTED in a build without the checks. */
+BD_API int bd_device_check_status(int32_t* code, int32_t* detail, int32_t reset);
+
 /* Human-readable name of a bd_status value. */
 BD_API const char* bd_status_string(int status);
 /* Text of the last CUDA error seen by a call of this thread (or ""). */

@@ -31,6 +31,14 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), n
 
 
+def test_checks_build_exports_the_same_symbols():
+    from decoding_bd_block_b200 import build
+    build.build()
+    checks = ctypes.CDLL(build.LIB_CHECKS)
+    for n in _declared():
+        assert hasattr(checks, n), n
+
+
 def test_binding_covers_header():
     from decoding_bd_block_b200 import bd
     assert sorted(bd.EXPORTED) == _declared()
