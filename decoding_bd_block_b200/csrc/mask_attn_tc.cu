@@ -76,7 +76,8 @@ __device__ __forceinline__ bool pair_visible(int i, int j, int L, int D) {
 __global__ void __launch_bounds__(kThreads, 1)
     mask_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, MaskArgs a) {
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_out, MaskArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -101,17 +102,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nq = (2 * w + 1 < a.G) ? 2 : 1;      // odd G: the last pair has one head
   const Span qs = span_of(qt, a.L, a.D);
 
-  if (threadIdx.x == 0) {
+  if (warp == 2) {
+    // The key tiles visible to this query tile, in order: one lane per tile
+    // (up to 63 tiles, two rounds), compacted with a ballot.
     int cnt = 0;
-    for (int kt = 0; kt < a.n_qt; ++kt) {
-      const int vis = tile_visibility(qs, span_of(kt, a.L, a.D), a.D);
+    for (int kt0 = 0; kt0 < a.n_qt; kt0 += 32) {
+      const int kt = kt0 + lane;
+      const int vis = kt < a.n_qt ? tile_visibility(qs, span_of(kt, a.L, a.D), a.D) : 0;
+      const uint32_t any = __ballot_sync(0xffffffffu, vis != 0);
       if (vis) {
-        kv_list[cnt] = static_cast<uint8_t>(kt);
-        kv_kind[cnt] = static_cast<uint8_t>(vis);
-        ++cnt;
+        const int at = cnt + __popc(any & ((1u << lane) - 1u));
+        kv_list[at] = static_cast<uint8_t>(kt);
+        kv_kind[at] = static_cast<uint8_t>(vis);
       }
+      cnt += __popc(any);
     }
-    kv_list[63] = static_cast<uint8_t>(cnt);
+    if (lane == 0) kv_list[63] = static_cast<uint8_t>(cnt);
+  }
+  if (threadIdx.x == 0) {
     tc::mbar_init(&q_full, 1);
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&kv_full[i], 1);
@@ -322,26 +330,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---------------------------------------------------------------- output
     if (ok && n_tiles > 0 && tc::mbar_wait_warp(&pv_done[t], (n_tiles - 1) & 1, a.status)) {
+      // O / l (bf16) of the warp's 32 rows goes through its 8 KB slice of the
+      // query tile's Q buffer (no MMA reads Q after the last P V), written in
+      // the 128-byte-swizzled layout of two (64 d x 32 rows) boxes, and out by
+      // TMA tile stores.
       tc::tc_fence_after();
       const int h = h0 + t;
       const uint32_t o_addr = tmem + lane_off + kColO + t * 128;
       const float inv = 1.f / l;
-      bf16* dst = a.out + ((static_cast<size_t>(row_base) + i) * a.Hq + h) * kD;
+      uint8_t* stg = smem + kOffQ + t * kQTileBytes + q * 8192;
+#pragma unroll 1
+      for (int dh = 0; dh < 2; ++dh) {  // 64 d per box
+        uint8_t* box = stg + dh * 4096;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t ov[32];
-        tc::tmem_ld_32x32b_x32(o_addr + cc * 32, ov);
-        tc::tmem_ld_wait();
-        uint32_t pkd[16];
+        for (int half = 0; half < 2; ++half) {
+          uint32_t ov[32];
+          tc::tmem_ld_32x32b_x32(o_addr + dh * 64 + half * 32, ov);
+          tc::tmem_ld_wait();
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
-          pkd[k] = tc::pack_bf16x2(__uint_as_float(ov[2 * k]) * inv,
-                                   __uint_as_float(ov[2 * k + 1]) * inv);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          d4[k] = make_uint4(pkd[4 * k], pkd[4 * k + 1], pkd[4 * k + 2], pkd[4 * k + 3]);
+          for (int k = 0; k < 4; ++k) {  // 8 bf16 = one 16-byte chunk
+            uint4 v;
+            v.x = tc::pack_bf16x2(__uint_as_float(ov[8 * k + 0]) * inv, __uint_as_float(ov[8 * k + 1]) * inv);
+            v.y = tc::pack_bf16x2(__uint_as_float(ov[8 * k + 2]) * inv, __uint_as_float(ov[8 * k + 3]) * inv);
+            v.z = tc::pack_bf16x2(__uint_as_float(ov[8 * k + 4]) * inv, __uint_as_float(ov[8 * k + 5]) * inv);
+            v.w = tc::pack_bf16x2(__uint_as_float(ov[8 * k + 6]) * inv, __uint_as_float(ov[8 * k + 7]) * inv);
+            const int chunk = half * 4 + k;
+            *reinterpret_cast<uint4*>(box + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = v;
+          }
+        }
       }
+      tc::fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        const int row = row_base + qt * kT + 32 * q;
+        tc::tma_store_3d(&tm_out, stg, 0, h, row);
+        tc::tma_store_3d(&tm_out, stg + 4096, 64, h, row);
+        tc::bulk_commit();
+        tc::bulk_wait_read<0>();
+      }
+      __syncwarp();
     }
   }
   tc::tc_fence_before();
@@ -368,14 +395,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows][H][128] bf16 viewed as (d, head, row): box = 128 rows of one head,
-// 64 d elements wide, 128-byte swizzle.
-bool make_tmap_heads(CUtensorMap* m, const void* base, uint64_t rows, uint32_t heads) {
+// [rows][H][128] bf16 viewed as (d, head, row): box = box_rows rows of one
+// head, 64 d elements wide, 128-byte swizzle (loads of 128-row tiles; tile
+// stores of 32 output rows).
+bool make_tmap_heads(CUtensorMap* m, const void* base, uint64_t rows, uint32_t heads,
+                     uint32_t box_rows = kT) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), heads, rows};
   const cuuint64_t strides[2] = {kD * 2, static_cast<cuuint64_t>(heads) * kD * 2};
-  const cuuint32_t box[3] = {64, 1, kT};
+  const cuuint32_t box[3] = {64, 1, box_rows};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -393,9 +422,9 @@ cudaError_t launch_mask_attn_tc(const bd_attn_shape& sh, const void* q, const vo
                                 int32_t* status, cudaStream_t st) {
   const int Hq = sh.n_heads_q, Hkv = sh.n_heads_kv;
   const uint64_t rows = static_cast<uint64_t>(n_seqs) * 2 * L;
-  CUtensorMap tm_q, tm_k, tm_v;
+  CUtensorMap tm_q, tm_k, tm_v, tm_out;
   if (!make_tmap_heads(&tm_q, q, rows, Hq) || !make_tmap_heads(&tm_k, k, rows, Hkv) ||
-      !make_tmap_heads(&tm_v, v, rows, Hkv))
+      !make_tmap_heads(&tm_v, v, rows, Hkv) || !make_tmap_heads(&tm_out, out, rows, Hq, 32))
     return cudaErrorInvalidValue;
   MaskArgs a{};
   a.L = L;
@@ -410,7 +439,7 @@ cudaError_t launch_mask_attn_tc(const bd_attn_shape& sh, const void* q, const vo
                        kSmemBytes);
   a.per_group = (a.G + 1) / 2;
   mask_attn_tc_kernel<<<dim3(a.per_group * Hkv, n_seqs, a.n_qt), kThreads, kSmemBytes, st>>>(
-      tm_q, tm_k, tm_v, a);
+      tm_q, tm_k, tm_v, tm_out, a);
   count_launches(1);
   return cudaGetLastError();
 }
