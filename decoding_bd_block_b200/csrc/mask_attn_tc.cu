@@ -132,6 +132,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc::fence_barrier_init();
     tc::fence_proxy_async();
+    // The query tiles do not depend on anything else: their loads start
+    // before the set-up barrier, overlapping the TMEM allocation.
+    tc::prefetch_tmap(&tm_q);
+    tc::mbar_arrive_expect_tx(&q_full, nq * kQTileBytes);
+    for (int t = 0; t < nq; ++t)
+      for (int dh = 0; dh < 2; ++dh)
+        tc::tma_load_3d(smem + kOffQ + t * kQTileBytes + dh * (kQTileBytes / 2), &tm_q, &q_full,
+                        dh * 64, h0 + t, n * 2 * a.L + qt * kT, tc::policy_evict_first());
   }
   if (warp == 1) tc::tmem_alloc(&tmem_slot, kTmemCols);
   tc::tc_fence_before();
@@ -145,19 +153,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
-      tc::prefetch_tmap(&tm_q);
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
     }
     const uint64_t pol_kv = tc::policy_evict_last();  // K/V tiles are re-read by other CTAs
-    const uint64_t pol_q = tc::policy_evict_first();
-    if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&q_full, nq * kQTileBytes);
-      for (int t = 0; t < nq; ++t)
-        for (int dh = 0; dh < 2; ++dh)
-          tc::tma_load_3d(smem + kOffQ + t * kQTileBytes + dh * (kQTileBytes / 2), &tm_q, &q_full,
-                          dh * 64, h0 + t, row_base + qt * kT, pol_q);
-    }
     int st = 0;
     uint32_t ph = 0;
     for (int j = 0; j < n_tiles; ++j) {
