@@ -244,20 +244,23 @@ __global__ void __launch_bounds__(256) attn_split_simt_kernel(
   }
 }
 
-// grid (Hq, batch), 256 threads: merge the chunks of one query head's 32
-// output rows.  Thread i owns row i / 8 and the D / 8 consecutive elements
-// (i % 8) * D / 8 ..; the eight threads of a row read its partial O rows as
-// contiguous 16-byte vectors.  Two passes over the chunks: the largest m
-// (base-2 exponent units), then the weighted sums of l and O.
+// grid (kBlock / 8, Hq, batch), 256 threads: merge the chunks of 8 output
+// rows of one query head, one warp per row.  Lane i holds the D / 32
+// consecutive elements i * D / 32 ..: a warp reads a partial O row as one
+// contiguous segment.  The chunks are taken eight at a time with all their
+// loads in flight and folded into a running (max, sum, O) in base-2 exponent
+// units, so a sequence of up to eight chunks costs one round trip to L2.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) attn_merge_kernel(const int32_t* __restrict__ n_blocks,
                                                          const float* __restrict__ part_o,
                                                          const float* __restrict__ part_ml,
                                                          T* __restrict__ out, int Hq, int ppc,
                                                          int max_chunks) {
-  constexpr int E = D / 8;  // elements per thread
-  const int h = blockIdx.x, s = blockIdx.y;
-  const int t = threadIdx.x / 8, d0 = (threadIdx.x % 8) * E;
+  constexpr int E = D / 32;  // elements per lane
+  static_assert(E == 2 || E == 4, "head_dim 64 or 128");
+  constexpr int kGroup = 8;  // chunks in flight
+  const int t = blockIdx.x * 8 + threadIdx.x / 32, h = blockIdx.y, s = blockIdx.z;
+  const int d0 = (threadIdx.x % 32) * E;
   griddep_wait();  // the split kernel's partials
   griddep_launch_dependents();
   const int total = max(n_blocks[s], 0) + 1;
@@ -265,34 +268,50 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const int32_t* __restri
   const int nch = min((total + ppc - 1) / ppc, max_chunks);
   const size_t base = (static_cast<size_t>(s) * Hq + h) * max_chunks;
   const float2* ml = reinterpret_cast<const float2*>(part_ml);
-  float M = -INFINITY;
-  for (int c = 0; c < nch; ++c) M = fmaxf(M, ml[(base + c) * kBlock + t].x);
-  float L = 0.f, acc[E];
+  float M = -INFINITY, L = 0.f, acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
-#pragma unroll 2
-  for (int c = 0; c < nch; ++c) {
-    const size_t r = (base + c) * kBlock + t;
-    const float2 v = ml[r];
-    const float w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
-    L = fmaf(v.y, w, L);
-    const float4* o = reinterpret_cast<const float4*>(part_o + r * D + d0);
+  for (int c0 = 0; c0 < nch; c0 += kGroup) {
+    float2 v[kGroup];
+    float o[kGroup][E];
 #pragma unroll
-    for (int e = 0; e < E / 4; ++e) {
-      const float4 x = o[e];
-      acc[4 * e + 0] = fmaf(x.x, w, acc[4 * e + 0]);
-      acc[4 * e + 1] = fmaf(x.y, w, acc[4 * e + 1]);
-      acc[4 * e + 2] = fmaf(x.z, w, acc[4 * e + 2]);
-      acc[4 * e + 3] = fmaf(x.w, w, acc[4 * e + 3]);
+    for (int u = 0; u < kGroup; ++u) {
+      v[u] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[u][e] = 0.f;
+      if (c0 + u < nch) {
+        const size_t r = (base + c0 + u) * kBlock + t;
+        v[u] = ml[r];
+        const float* src = part_o + r * D + d0;
+        if constexpr (E == 4) {
+          const float4 x = *reinterpret_cast<const float4*>(src);
+          o[u][0] = x.x, o[u][1] = x.y, o[u][2] = x.z, o[u][3] = x.w;
+        } else {
+          const float2 x = *reinterpret_cast<const float2*>(src);
+          o[u][0] = x.x, o[u][1] = x.y;
+        }
+      }
     }
+    float Mn = M;
+#pragma unroll
+    for (int u = 0; u < kGroup; ++u) Mn = fmaxf(Mn, v[u].x);
+    const float sc = M == -INFINITY ? 0.f : exp2f(M - Mn);
+    L *= sc;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] *= sc;
+#pragma unroll
+    for (int u = 0; u < kGroup; ++u) {
+      const float w = v[u].x == -INFINITY ? 0.f : exp2f(v[u].x - Mn);
+      L = fmaf(v[u].y, w, L);
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(o[u][e], w, acc[e]);
+    }
+    M = Mn;
   }
   const float inv = 1.f / L;
-  T res[E];
+  T* dst = out + ((static_cast<size_t>(s) * kBlock + t) * Hq + h) * D + d0;
 #pragma unroll
-  for (int e = 0; e < E; ++e) res[e] = from_f32<T>(acc[e] * inv);
-  uint4* dst = reinterpret_cast<uint4*>(out + ((static_cast<size_t>(s) * kBlock + t) * Hq + h) * D + d0);
-#pragma unroll
-  for (int e = 0; e < static_cast<int>(E * sizeof(T) / 16); ++e) dst[e] = reinterpret_cast<const uint4*>(res)[e];
+  for (int e = 0; e < E; ++e) dst[e] = from_f32<T>(acc[e] * inv);
 }
 
 // -------------------------------------------------------------- host side
@@ -384,7 +403,7 @@ static cudaError_t launch_attn_t(const bd_attn_shape& sh, const bd_kv_cache& c, 
                        reinterpret_cast<int32_t*>(w + p.off_status), st);
     if (e != cudaSuccess) return e;
     if (p.max_chunks > 1) {
-      e = launch_pdl(attn_merge_kernel<T, D>, dim3(sh.n_heads_q, c.batch), dim3(256), 0, st,
+      e = launch_pdl(attn_merge_kernel<T, D>, dim3(kBlock / 8, sh.n_heads_q, c.batch), dim3(256), 0, st,
                      c.n_blocks, part_o, part_ml, static_cast<T*>(out), sh.n_heads_q,
                      p.pages_per_chunk, p.max_chunks);
       if (e != cudaSuccess) return e;
@@ -400,7 +419,7 @@ static cudaError_t launch_attn_t(const bd_attn_shape& sh, const bd_kv_cache& c, 
       ws_blk, part_o, part_ml, static_cast<T*>(out), sh.n_heads_q, sh.n_heads_kv,
       p.pages_per_chunk, p.max_chunks);
   if (p.max_chunks > 1)
-    attn_merge_kernel<T, D><<<dim3(sh.n_heads_q, c.batch), 256, 0, st>>>(
+    attn_merge_kernel<T, D><<<dim3(kBlock / 8, sh.n_heads_q, c.batch), 256, 0, st>>>(
         c.n_blocks, part_o, part_ml, static_cast<T*>(out), sh.n_heads_q, p.pages_per_chunk,
         p.max_chunks);
   count_launches(p.max_chunks > 1 ? 2 : 1);

@@ -280,38 +280,74 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       uint32_t sr[128];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc)
-        tc::tmem_ld_32x32b_x32(sbuf + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
-      tc::tmem_ld_wait();
-      if (valid < kKeys) {  // warp-uniform: only the last stage of a chunk can be partial
-#pragma unroll
-        for (int k = 32; k < 128; ++k)
-          if (k >= valid) sr[k] = __float_as_uint(-INFINITY);
-      }
-      float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int k = 0; k < 128; k += 2)
-        mk[(k >> 1) & 3] = tc::fmax3(mk[(k >> 1) & 3], __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
-      const float mt = fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])) * scale;
-      const float m_new = fmaxf(m, mt);
-      const bool rescale = (m == -INFINITY) || (m_new - m > kRescaleThreshold);
       float alpha = 1.f;
-      if (rescale) {
-        alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
-        m = m_new;
-      }
-      const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(-m, -m);
-      float2 rk[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      bool rescale = false;
+      float2 rk[2];
+      int jmax;
+      // The 16 pairs of 32-column chunk cc: p = 2^(s * scale - m) in paired
+      // fp32 arithmetic, a quarter of the pairs on the FMA pipe, the rest on
+      // MUFU; packed in place, sr[k] <- (p_2k, p_2k+1).
+      auto exps = [&](int cc) {
+        const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(-m, -m);
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {  // packs in place: sr[k] <- (p_2k, p_2k+1)
-        // paired fp32 arithmetic; a quarter of the pairs' exponentials on the
-        // FMA pipe, the rest on MUFU (the MUFU unit bounds this loop)
-        const float2 x = ffma2(make_float2(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])),
-                               sc2, nm2);
-        const float2 e = kPolyPair(k) ? poly_exp2x2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
-        rk[k & 1] = fadd2(rk[k & 1], e);
-        sr[k] = tc::pack_bf16x2(e.x, e.y);
+        for (int k = 16 * cc; k < 16 * cc + 16; ++k) {
+          const float2 x = ffma2(make_float2(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])),
+                                 sc2, nm2);
+          const float2 e = kPolyPair(k) ? poly_exp2x2(x, jmax) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          rk[k & 1] = fadd2(rk[k & 1], e);
+          sr[k] = tc::pack_bf16x2(e.x, e.y);
+        }
+      };
+      // A full stage after the first: the exponentials are taken against the
+      // running max m as it stands, without a max pass, and each 32-column
+      // TMEM load of S overlaps the exponentials of the chunk before.  That
+      // equals the max-pass result whenever no score of the stage exceeds m
+      // by more than kRescaleThreshold (the only case in which the max pass
+      // moves m): a stage sum of exponentials <= 2^8 and a largest integer
+      // part <= 8 among the polynomial pairs prove it.  Otherwise, and at the
+      // first or a partial stage, the max pass runs and the exponentials are
+      // taken again (S is still in TMEM).
+      bool done = false;
+      if (j > 0 && valid == kKeys) {  // warp-uniform
+        rk[0] = rk[1] = make_float2(0.f, 0.f);
+        jmax = 0;
+        tc::tmem_ld_32x32b_x32(sbuf, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          tc::tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+          if (cc < 3)
+            tc::tmem_ld_32x32b_x32(sbuf + (cc + 1) * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * (cc + 1)]));
+          exps(cc);
+        }
+        const float sum = (rk[0].x + rk[0].y) + (rk[1].x + rk[1].y);
+        static_assert(kRescaleThreshold == 8.f, "the bounds below are 2^8 and 8");
+        done = !__any_sync(0xffffffffu, !(sum <= 256.f) || jmax > 8);
+      }
+      if (!done) {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          tc::tmem_ld_32x32b_x32(sbuf + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+        tc::tmem_ld_wait();
+        if (valid < kKeys) {  // warp-uniform: only the last stage of a chunk can be partial
+#pragma unroll
+          for (int k = 32; k < 128; ++k)
+            if (k >= valid) sr[k] = __float_as_uint(-INFINITY);
+        }
+        float mk[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int k = 0; k < 128; k += 2)
+          mk[(k >> 1) & 3] = tc::fmax3(mk[(k >> 1) & 3], __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
+        const float mt = fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])) * scale;
+        const float m_new = fmaxf(m, mt);
+        rescale = (m == -INFINITY) || (m_new - m > kRescaleThreshold);
+        if (rescale) {
+          alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
+          m = m_new;
+        }
+        rk[0] = rk[1] = make_float2(0.f, 0.f);
+        jmax = 0;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) exps(cc);
       }
       l = l * alpha + ((rk[0].x + rk[0].y) + (rk[1].x + rk[1].y));
       // TMEM accesses are warp-collective, so the warp rescales together when

@@ -92,6 +92,25 @@ __device__ __forceinline__ float2 poly_exp2x2(float2 x) {
                      __int_as_float(__float_as_int(p.y) + jy * (1 << 23)));
 }
 
+// The same, also raising jmax to the larger integer part round(x) of the
+// pair (the polynomial's result is 2^x only while that is below 128).
+__device__ __forceinline__ float2 poly_exp2x2(float2 x, int& jmax) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = fadd2(x, make_float2(12582912.f, 12582912.f));
+  const int jx = __float_as_int(t.x) - 0x4B400000, jy = __float_as_int(t.y) - 0x4B400000;
+  jmax = __vimax3_s32(jmax, jx, jy);
+  const float2 u = fadd2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = ffma2(u, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(make_float2(0.009570101434f, 0.009570101434f), f,
+                   make_float2(0.05591786028f, 0.05591786028f));
+  p = ffma2(p, f, make_float2(0.2402474484f, 0.2402474484f));
+  p = ffma2(p, f, make_float2(0.6931218147f, 0.6931218147f));
+  p = ffma2(p, f, make_float2(0.9999992614f, 0.9999992614f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + jx * (1 << 23)),
+                     __int_as_float(__float_as_int(p.y) + jy * (1 << 23)));
+}
+
 // ------------------------------------------- programmatic dependent launch
 // A kernel launched with launch_pdl() may start while the previous kernel of
 // the stream is still running: it must call griddep_wait() before it reads

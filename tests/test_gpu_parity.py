@@ -171,6 +171,34 @@ def test_block_attn_growing_scores_vs_fp64_oracle():
     assert max(float(np.abs(got[s] - ref[s]).max()) for s in ref) <= ATOL["bf16"]
 
 
+def test_block_attn_score_spikes():
+    """Single keys 100x larger than the rest, deep inside the cache: their
+    scores exceed the running max by up to several hundred (base 2), far past
+    the range of the FMA-pipe exponential.  Placed at key columns 6, 7 (mod 8)
+    of a 128-key stage they fall on the polynomial pairs, elsewhere on the
+    MUFU pairs; every row must still match the oracle with bf16 operands."""
+    cfg = dataclasses.replace(W.QWEN7B_RAGGED, name="bf16_spikes", batch=2, prefix_range=(),
+                              prefix_tokens=(3072, 1504), seed=104)
+    a = W.make_attn_inputs(cfg)
+    spikes = {0: (1030, 1500, 2055), 1: (700, 1270)}
+    for s, toks in spikes.items():
+        k = W.f32_from_bf16_bits(a["prefix_k"][s])
+        for t in toks:
+            k[t] *= 100.0
+        a["prefix_k"][s] = W.bf16_bits_from_f32(k)
+    from decoding_bd_block_b200.step import DecodeStep
+    step = DecodeStep(cfg, a, None)
+    step.run_attn()
+    torch.cuda.synchronize()
+    got = step.out.float().cpu().numpy()
+    emu = bf16_storage_block_attn(cfg, a)
+    for s in emu:
+        assert np.isfinite(got[s]).all()
+        err = float(np.abs(got[s] - emu[s]).max())
+        print(f"seq {s}: vs bf16-operand oracle {err:.3e}")
+        assert err <= ATOL["bf16"], (s, err)
+
+
 def test_block_attn_repeatable_and_after_commit():
     # The block attention reads n_blocks on the device: commit the current
     # block, attend again with a new block, compare with the oracle.
