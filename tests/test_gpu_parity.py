@@ -94,6 +94,12 @@ ATTN_CASES = [
     # G = 1: 32 query rows per CTA
     dataclasses.replace(W.QWEN15B_STEP, name="bf16_g1", n_heads_q=4, n_heads_kv=4,
                         prefix_tokens=(64,), seed=102),
+    # CTA pairs: G = 8 fills both 128-row halves; G = 5 leaves three padding
+    # warps in the second
+    dataclasses.replace(W.QWEN15B_STEP, name="bf16_g8_pair_full", n_heads_q=16, n_heads_kv=2,
+                        batch=2, prefix_tokens=(992, 4128), seed=105),
+    dataclasses.replace(W.QWEN15B_STEP, name="bf16_g5_pair_pad", n_heads_q=10, n_heads_kv=2,
+                        batch=2, prefix_tokens=(32, 2400), seed=106),
 ]
 
 
