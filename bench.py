@@ -233,21 +233,30 @@ def oracle_caches(cfg, a_in, seqs=None):
 def oracle_step_sample(cfg, a_in, s_in, frac: float, tau: float, S: int, caches=None):
     """One oracle step on a bounded sample: block attention of the sequences
     in ``caches`` (all of them when None), and the LM-head statistics /
-    selection over the first `frac` of the vocabulary.  Returns the
-    masked-position equivalents scored (frac x masked positions)."""
+    selection over the first `frac` of the vocabulary.  Returns
+    (attention seconds, LM-head seconds, vocabulary fraction actually used)."""
     import oracle as O
+    t0 = time.perf_counter()
     if a_in is not None:
         caches = oracle_caches(cfg, a_in) if caches is None else caches
         for s, c in caches.items():
             O.block_attn_seq(c.k[0], c.v[0], O.widen(a_in["q"][s], cfg.dtype),
                              O.widen(a_in["k_blk"][s], cfg.dtype),
                              O.widen(a_in["v_blk"][s], cfg.dtype), cfg.rope_theta)
+    t1 = time.perf_counter()
     if s_in is None:
-        return 0.0
+        return t1 - t0, 0.0, 1.0
     Vs = max(1, int(round(cfg.vocab * frac)))
-    r = O.confidence_select(s_in["h"], s_in["h_prev"], s_in["W"][:Vs], s_in["masked_bits"], tau, S,
-                            s_in["tokens"], cfg.dtype)
-    return r["n_scored"] * Vs / cfg.vocab
+    O.confidence_select(s_in["h"], s_in["h_prev"], s_in["W"][:Vs], s_in["masked_bits"], tau, S,
+                        s_in["tokens"], cfg.dtype)
+    return t1 - t0, time.perf_counter() - t1, Vs / cfg.vocab
+
+
+def full_step_seconds(parts):
+    """Whole-step seconds estimated from sampled steps [(attention s, LM-head s,
+    vocabulary fraction)]: the attention as timed, the LM-head time scaled to
+    the full vocabulary (it is linear in the vocabulary rows)."""
+    return sum(ta + tl / f for ta, tl, f in parts) / len(parts)
 
 
 def blas_threads():
@@ -270,9 +279,7 @@ def cpu_baseline(cfg, a_in, s_in, tau, S, budget_s, got=None):
     step sized to about budget_s, and no parity block."""
     import platform
     caches = oracle_caches(cfg, a_in) if a_in is not None else None
-    t0 = time.perf_counter()
-    oracle_step_sample(cfg, a_in, s_in, 0.02, tau, S, caches)  # probe: 2% of the vocab
-    probe = max(time.perf_counter() - t0, 1e-3)
+    probe = max(sum(oracle_step_sample(cfg, a_in, s_in, 0.02, tau, S, caches)[:2]), 1e-3)  # 2% of the vocab
     cpu = platform.processor() or platform.machine()
     n_pos = s_in["n_scored"] if s_in else 0
     if s_in is None or probe * 50 <= 3 * budget_s:  # (attention only: the probe was a whole step)
@@ -289,17 +296,16 @@ def cpu_baseline(cfg, a_in, s_in, tau, S, budget_s, got=None):
                            + f"; fp64 numpy on {cpu}")}
         return base, (parity_block(cfg, ref, got, tau, S) if got is not None else None)
     frac = float(min(1.0, max(0.02, 0.02 * budget_s / probe / 2)))
-    scored, t_total, n = 0.0, 0.0, 0
-    while t_total < budget_s * 0.5 or n == 0:
-        t0 = time.perf_counter()
-        scored += oracle_step_sample(cfg, a_in, s_in, frac, tau, S, caches)
-        t_total += time.perf_counter() - t0
-        n += 1
-    return {"value": scored / t_total, "unit": "masked positions scored/s", "cores": blas_threads(),
-            "kind": "oracle",
-            "sample": (f"{n} oracle step(s) of workload {cfg.name}: full block attention + "
-                       f"LM-head statistics and selection over {frac:.1%} of the vocabulary "
-                       f"({frac:.3f} x {n_pos} masked positions per step); fp64 numpy on {cpu}")}, None
+    parts, t_total = [], 0.0
+    while t_total < budget_s * 0.5 or not parts:
+        parts.append(oracle_step_sample(cfg, a_in, s_in, frac, tau, S, caches))
+        t_total += sum(parts[-1][:2])
+    return {"value": n_pos / full_step_seconds(parts), "unit": "masked positions scored/s",
+            "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"{len(parts)} oracle step(s) of workload {cfg.name}: full block attention + "
+                       f"LM-head statistics and selection over {parts[0][2]:.1%} of the vocabulary, "
+                       f"the LM-head time scaled to the full vocabulary ({n_pos} masked positions "
+                       f"per step); fp64 numpy on {cpu}")}, None
 
 
 def oracle_full_step(cfg, a_in, s_in, tau, S, caches):
@@ -417,23 +423,18 @@ def run_reference(args, cfg, tau, S):
         return
     s_in["n_scored"] = int(sum(bin(int(b)).count("1") for b in s_in["masked_bits"]))
     caches = oracle_caches(cfg, a_in)
-    t0 = time.perf_counter()
-    oracle_step_sample(cfg, a_in, s_in, 0.02, tau, S, caches)
-    probe = max(time.perf_counter() - t0, 1e-3)
+    probe = max(sum(oracle_step_sample(cfg, a_in, s_in, 0.02, tau, S, caches)[:2]), 1e-3)
     frac = float(min(1.0, max(0.002, 0.02 * reference_budget(args) / probe)))
     for _ in range(args.warmup):
         oracle_step_sample(cfg, a_in, s_in, frac, tau, S, caches)
-    scored, t = 0.0, 0.0
-    for _ in range(args.steps):
-        t0 = time.perf_counter()
-        scored += oracle_step_sample(cfg, a_in, s_in, frac, tau, S, caches)
-        t += time.perf_counter() - t0
+    parts = [oracle_step_sample(cfg, a_in, s_in, frac, tau, S, caches) for _ in range(args.steps)]
+    t_step = full_step_seconds(parts)
     line = reference_line(
         args, cfg.name, "masked positions scored/s per denoise step", "masked positions scored/s",
-        scored / t, t, {"batch": cfg.batch, "tau": tau, "sub_block": S,
-                        "vocab_fraction_per_step": frac},
-        f"each step: full block attention + LM-head statistics over {frac:.2%} of the "
-        f"vocabulary of workload {cfg.name}")
+        s_in["n_scored"] / t_step, t_step * args.steps,
+        {"batch": cfg.batch, "tau": tau, "sub_block": S, "vocab_fraction_per_step": parts[0][2]},
+        f"each step: full block attention + LM-head statistics over {parts[0][2]:.2%} of the "
+        f"vocabulary of workload {cfg.name}, the LM-head time scaled to the full vocabulary")
     print(json.dumps(line), flush=True)
 
 
