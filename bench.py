@@ -177,6 +177,25 @@ def gpu_uuid(dev):
         return None
 
 
+class L2Flush:
+    """The L2 flush between timed steps: write a buffer larger than L2, which
+    evicts every line of the previous step, then read a second one, so that L2
+    is left holding clean lines of unrelated data rather than dirty ones that
+    the next step would write back to HBM while it runs (a step in a serving
+    loop does not start behind a 256 MB memset)."""
+    DESCRIPTION = (f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write, then a "
+                   f"{L2_FLUSH_BYTES >> 20} MB read so that no dirty line is left)")
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -521,11 +540,11 @@ def run_ours(args, cfg, tau, S, dist: Dist):
         # the kernels score only the candidates: count those as the units
         step.active_only = True
         step.n_scored = sum(bin(active_bits(int(b), S)).count("1") for b in step.masked_host)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step.run(tau, S)
     torch.cuda.synchronize(dev)
     # Kernels one step launches (counted on an eager step), then the step's
@@ -541,7 +560,7 @@ def run_ours(args, cfg, tau, S, dist: Dist):
     sel_launches = per_step - (n1 - n0)
     graphs = None if args.eager else step.capture(tau, S, parts=("step", "attn", "select"))
     for _ in range(2):
-        flush.zero_()
+        flush()
         if graphs:
             graphs["step"].replay()
         else:
@@ -561,7 +580,7 @@ def run_ours(args, cfg, tau, S, dist: Dist):
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
     for i in range(K):
-        flush.zero_()
+        flush()
         ev[i][0].record(stream)
         if graphs:
             graphs["step"].replay()
@@ -582,7 +601,7 @@ def run_ours(args, cfg, tau, S, dist: Dist):
     n_bd = max(10, K // 4)
     evb = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_bd)]
     for i in range(n_bd):
-        flush.zero_()
+        flush()
         evb[i][0].record(stream)
         if step.attn:
             graphs["attn"].replay() if graphs else step.run_attn()
@@ -648,7 +667,7 @@ def run_ours(args, cfg, tau, S, dist: Dist):
                    "prefix_tokens": [int(x) for x in a_in["prefix_len"]],
                    "hidden": cfg.hidden, "vocab": cfg.vocab, "tau": tau, "sub_block": S,
                    "masked_positions_per_step": n_scored,
-                   "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
+                   "l2": L2Flush.DESCRIPTION,
                    "parallelism": f"replicas x{dist.world} (independent batches)",
                    "launch": "eager" if args.eager else "CUDA graph replay of the C-ABI calls"},
         "breakdown_ms": {"bd_block_attn": float(np.mean(t_attn)),
@@ -706,7 +725,7 @@ def measure_e2e(step, cfg, tau, S, flush, dev, dist, K, graph=None):
             if i >= 1:
                 copy_stream.wait_event(consumed[1 - b])
             upload(1 - b)
-        flush.zero_()
+        flush()
         ev[i][0].record(stream)
         stream.wait_event(uploaded[b])
         step.arena[:step.in_bytes].copy_(staging[b], non_blocking=True)
@@ -748,11 +767,11 @@ def run_mask_attn(args, cfg, dist: Dist):
     q, k, v = (to_device(t[x], cfg.dtype, dev) for x in ("q", "k", "v"))
     out = torch.empty_like(q)
     shape = bd.make_shape(cfg.n_heads_q, cfg.n_heads_kv, cfg.head_dim, cfg.dtype)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
     call = lambda: bd.bd_block_mask_attn(shape, q, k, v, out, cfg.n_seqs, cfg.L, cfg.block)
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         call()
     torch.cuda.synchronize(dev)
     K = args.steps
@@ -763,7 +782,7 @@ def run_mask_attn(args, cfg, dist: Dist):
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
     for i in range(K):
-        flush.zero_()
+        flush()
         ev[i][0].record(stream)
         call()
         ev[i][1].record(stream)
@@ -786,7 +805,7 @@ def run_mask_attn(args, cfg, dist: Dist):
         "config": {"workload": cfg.name, "views": cfg.n_seqs, "L": cfg.L, "block": cfg.block,
                    "n_heads_q": cfg.n_heads_q, "n_heads_kv": cfg.n_heads_kv,
                    "head_dim": cfg.head_dim, "allowed_pairs_per_view_head": pairs,
-                   "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)"},
+                   "l2": L2Flush.DESCRIPTION},
         "roofline": {"kernel": "bd_block_mask_attn", "bound": "tensor", "achieved": ach,
                      "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
                      "traffic": recorded_traffic("mask_attn"),
@@ -818,12 +837,12 @@ def run_masked_ce(args, cfg, dist: Dist):
     ns = torch.zeros(1, dtype=torch.int32, device=dev)
     ws = torch.empty(bd.bd_masked_ce_workspace_size(cfg.dtype, N, L, cfg.hidden, cfg.vocab),
                      dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
     call = lambda: bd.bd_masked_ce(cfg.dtype, N, L, cfg.hidden, cfg.vocab, h, w, tg, mb, loss, ls,
                                    ns, ws)
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         call()
     torch.cuda.synchronize(dev)
     count = int(ns.item())
@@ -835,7 +854,7 @@ def run_masked_ce(args, cfg, dist: Dist):
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
     for i in range(K):
-        flush.zero_()
+        flush()
         ev[i][0].record(stream)
         call()
         ev[i][1].record(stream)
@@ -858,7 +877,7 @@ def run_masked_ce(args, cfg, dist: Dist):
         "config": {"workload": cfg.name, "sequences": N, "L": L, "hidden": cfg.hidden,
                    "vocab": cfg.vocab, "scored_positions": count,
                    "mean_loss": float(ls.item()) / max(count, 1),
-                   "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)"},
+                   "l2": L2Flush.DESCRIPTION},
         "roofline": {"kernel": "bd_masked_ce (LM head on tcgen05; whole call timed)",
                      "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                      "frac": ach / peak, "traffic": recorded_traffic("masked_ce"),
