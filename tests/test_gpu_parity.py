@@ -367,6 +367,17 @@ def test_mask_attn_parity_small(L, D, dtype, d, Hq, Hkv):
     assert float(np.abs(got - ref).max()) <= ATOL[dtype]
 
 
+def test_mask_attn_many_items_per_cta():
+    """More work items than SMs (4 query tiles x 40 views x 4 head pairs =
+    640 items, about four per persistent CTA, single-head pairs among them):
+    every row of every view against the oracle."""
+    cfg, t = _mask_case(256, 32, "bf16", n=20, d=128, Hq=6, Hkv=2, seed=7)
+    got = _run_mask(cfg, t)
+    ref = O.mask_attn(O.widen(t["q"], "bf16"), O.widen(t["k"], "bf16"), O.widen(t["v"], "bf16"),
+                      cfg.L, cfg.block)
+    assert float(np.abs(got - ref).max()) <= ATOL["bf16"]
+
+
 def test_mask_attn_full_size_sampled():
     cfg = W.MASK_ATTN
     t = W.make_mask_attn_inputs(cfg)
