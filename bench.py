@@ -50,6 +50,9 @@ def parse_args(argv=None):
     ap.add_argument("--tau", type=float, default=None)
     ap.add_argument("--sub-block", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shared-clean", action="store_true",
+                    help="mask attention: compute each sample's clean rows once for all its views "
+                         "(bd_block_mask_attn_views)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--active-only", action="store_true",
@@ -754,6 +757,14 @@ def mask_pairs(L: int, D: int) -> int:
     return D * D * (n * n + n)
 
 
+def mask_clean_pairs(L: int, D: int) -> int:
+    """The clean queries' share of mask_pairs: (b + 1) D^2 for block b,
+    D^2 n (n + 1) / 2 in all.  They see clean keys only, so they are the same
+    in every view of a sample."""
+    n = L // D
+    return D * D * n * (n + 1) // 2
+
+
 def run_mask_attn(args, cfg, dist: Dist):
     """bd_block_mask_attn on the training-forward workload (2L x 2L mask)."""
     import torch
@@ -769,7 +780,11 @@ def run_mask_attn(args, cfg, dist: Dist):
     shape = bd.make_shape(cfg.n_heads_q, cfg.n_heads_kv, cfg.head_dim, cfg.dtype)
     flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
-    call = lambda: bd.bd_block_mask_attn(shape, q, k, v, out, cfg.n_seqs, cfg.L, cfg.block)
+    if args.shared_clean:
+        call = lambda: bd.bd_block_mask_attn_views(shape, q, k, v, out, cfg.n_seqs, cfg.views,
+                                                   cfg.L, cfg.block)
+    else:
+        call = lambda: bd.bd_block_mask_attn(shape, q, k, v, out, cfg.n_seqs, cfg.L, cfg.block)
     for _ in range(args.warmup):
         flush()
         call()
@@ -794,6 +809,9 @@ def run_mask_attn(args, cfg, dist: Dist):
                                         float(np.mean([e[0].elapsed_time(e[1]) for e in ev])), dev)
     pairs = mask_pairs(cfg.L, cfg.block)
     flop = 4.0 * cfg.head_dim * cfg.n_heads_q * pairs * cfg.n_seqs
+    if args.shared_clean:  # each sample's clean rows computed once, for all of its views
+        flop -= (4.0 * cfg.head_dim * cfg.n_heads_q * mask_clean_pairs(cfg.L, cfg.block)
+                 * (cfg.n_seqs - cfg.samples))
     peaks, peak_kind = measured_peaks()
     peak = float(peaks.get("bf16_tflops", 1590.0))
     ach = flop / (ms / 1e3) / 1e12
@@ -805,10 +823,13 @@ def run_mask_attn(args, cfg, dist: Dist):
         "config": {"workload": cfg.name, "views": cfg.n_seqs, "L": cfg.L, "block": cfg.block,
                    "n_heads_q": cfg.n_heads_q, "n_heads_kv": cfg.n_heads_kv,
                    "head_dim": cfg.head_dim, "allowed_pairs_per_view_head": pairs,
+                   "clean_rows": (f"computed once per sample for its {cfg.views} views"
+                                  if args.shared_clean else "computed for every view"),
                    "l2": L2Flush.DESCRIPTION},
         "roofline": {"kernel": "bd_block_mask_attn", "bound": "tensor", "achieved": ach,
                      "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-                     "traffic": recorded_traffic("mask_attn"),
+                     "traffic": recorded_traffic("mask_attn_views" if args.shared_clean
+                                                 else "mask_attn"),
                      "algorithmic_flop_per_launch": flop, "peak_source": peak_kind},
         "gpu_launches": int(launches),
         "clocks": clocks,

@@ -24,7 +24,7 @@ EXPORTED = ("bd_cache_commit", "bd_block_attn_workspace_size", "bd_block_attn",
             "bd_block_mask_attn", "bd_status_string", "bd_last_cuda_error_string",
             "bd_kernel_launches", "bd_confidence_select_noalloc", "bd_confidence_select_active",
             "bd_masked_ce_workspace_size", "bd_masked_ce", "bd_eval_exp2",
-            "bd_device_check_status")
+            "bd_device_check_status", "bd_block_mask_attn_views")
 BD_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 if not os.path.exists(_LIB_PATH):
@@ -69,6 +69,8 @@ _SIGS = {
     "bd_confidence_select": [_I, _I, _I, _I, _P, _P, _P, _P, ctypes.c_float, _I, _P, _P, _P, _P,
                              _P, ctypes.c_size_t, _P],
     "bd_block_mask_attn": [ctypes.POINTER(bd_attn_shape), _P, _P, _P, _P, _I, _I, _I, _P],
+    "bd_block_mask_attn_views": [ctypes.POINTER(bd_attn_shape), _P, _P, _P, _P, _I, _I, _I, _I,
+                                 _P],
     "bd_confidence_select_noalloc": [_I, _I, _I, _I, _P, _P, _P, _P, ctypes.c_float, _I, _P, _P,
                                      _P, _P, _P],
     "bd_confidence_select_active": [_I, _I, _I, _I, _P, _P, _P, _P, ctypes.c_float, _I, _P, _P,
@@ -238,6 +240,15 @@ def bd_block_mask_attn(shape: bd_attn_shape, q, k, v, out, n_seqs, L, block, str
     _check("bd_block_mask_attn", _lib.bd_block_mask_attn(
         ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out), int(n_seqs), int(L),
         int(block), _stream(stream)))
+
+
+def bd_block_mask_attn_views(shape: bd_attn_shape, q, k, v, out, n_seqs, views, L, block,
+                             stream=None):
+    """bd_block_mask_attn for entries in groups of `views` views of one sample
+    whose clean halves are equal (see include/bd.h)."""
+    _check("bd_block_mask_attn_views", _lib.bd_block_mask_attn_views(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out), int(n_seqs), int(views),
+        int(L), int(block), _stream(stream)))
 
 
 def bd_eval_exp2(x, y_poly, y_pair, y_mufu, stream=None):

@@ -12,6 +12,7 @@
 //                  (max, sum, O) per query row, in base-2 exponent units;
 //   3. attn_merge  combines the chunks' (m, l, O) per row.
 #include "bd_common.cuh"
+#include "mask_attn.cuh"
 
 namespace bd {
 
@@ -525,8 +526,14 @@ static cudaError_t launch_mask_t(const bd_attn_shape& sh, const void* q, const v
 cudaError_t launch_block_mask_attn(const bd_attn_shape& sh, const void* q, const void* k,
                                    const void* v, void* out, int n_seqs, int L, int block,
                                    cudaStream_t st) {
+  return launch_block_mask_attn_views(sh, q, k, v, out, n_seqs, 1, L, block, st);
+}
+
+cudaError_t launch_block_mask_attn_views(const bd_attn_shape& sh, const void* q, const void* k,
+                                         const void* v, void* out, int n_seqs, int views, int L,
+                                         int block, cudaStream_t st) {
   if (mask_attn_tc_supported(sh, L))
-    return launch_mask_attn_tc(sh, q, k, v, out, n_seqs, L, block, nullptr, st);
+    return launch_mask_attn_tc_views(sh, q, k, v, out, n_seqs, views, L, block, nullptr, st);
   const bool b = sh.dtype == BD_BF16;
   if (sh.head_dim == 64)
     return b ? launch_mask_t<bf16, 64>(sh, q, k, v, out, n_seqs, L, block, st)

@@ -8,6 +8,7 @@
 #include <nvtx3/nvToolsExt.h>
 
 #include "bd_common.cuh"
+#include "mask_attn.cuh"
 
 namespace bd {
 static std::atomic<long long> g_launches{0};
@@ -291,6 +292,21 @@ int bd_block_mask_attn(const bd_attn_shape* sh, const void* q, const void* k, co
   if (L % bd::kBlock != 0 || 2LL * L / bd::kBlock > 2147483647LL) return BD_ERR_UNSUPPORTED;
   return cuda_status(bd::launch_block_mask_attn(*sh, q, k, v, out, n_seqs, L, block,
                                                 static_cast<cudaStream_t>(stream)));
+}
+
+int bd_block_mask_attn_views(const bd_attn_shape* sh, const void* q, const void* k,
+                             const void* v, void* out, int32_t n_seqs, int32_t views, int32_t L,
+                             int32_t block, void* stream) {
+  NvtxRange nvtx_range("bd_block_mask_attn_views");
+  int st = check_shape(sh);
+  if (st) return st;
+  if (!q || !k || !v || !out || n_seqs <= 0 || n_seqs > 65535 || L <= 0 || block <= 0)
+    return BD_ERR_INVALID_ARG;
+  if (views <= 0 || n_seqs % views != 0) return BD_ERR_INVALID_ARG;
+  if (L % block != 0) return BD_ERR_INVALID_ARG;
+  if (L % bd::kBlock != 0 || 2LL * L / bd::kBlock > 2147483647LL) return BD_ERR_UNSUPPORTED;
+  return cuda_status(bd::launch_block_mask_attn_views(*sh, q, k, v, out, n_seqs, views, L, block,
+                                                      static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -16,7 +16,14 @@
 // S_t = Q_t K^T (SS MMA); one thread per query row runs the base-2 online
 // softmax with lazy rescaling, as in attn_tc.cu.  Every key of a row is
 // seen within one item, so O / l goes straight to the output.
+//
+// Views that share a sample: the two complementary-mask views of one
+// training sample differ only in their noisy stream; the clean stream x_0,
+// and with it every clean query's output (clean queries see clean keys
+// only), is the same.  With views > 1 the clean query tiles of a sample are
+// computed once and stored into the rows of each of its views.
 #include "bd_common.cuh"
+#include "mask_attn.cuh"
 #include "tc_common.cuh"
 
 namespace bd {
@@ -40,8 +47,10 @@ struct MaskArgs {
   int L, D, Hq, Hkv, G;
   int n_qt;       // 2L / 128
   int per_group;  // query-head pairs per KV group: ceil(G / 2)
-  int n_seqs;     // views
-  int n_items;    // n_qt x n_seqs x per_group x Hkv work items
+  int n_seqs;     // entries (samples x views)
+  int views;      // consecutive entries that share one clean stream
+  int n_samples;  // n_seqs / views
+  int n_items;    // n_qt / 2 x (n_seqs + n_samples) x per_group x Hkv work items
   bf16* out;
   int32_t* status;
 };
@@ -79,7 +88,7 @@ __device__ __forceinline__ bool pair_visible(int i, int j, int L, int D) {
 }
 
 // One work item = (128-row query tile, pair of query heads of one KV group,
-// view): the unit the kernel used to give each CTA.  The grid is one
+// entry): the unit the kernel used to give each CTA.  The grid is one
 // persistent CTA per SM; CTA c takes items c, then 2G-1-c, then 2G+c, ...
 // (G CTAs, a snake over the items ranked heaviest first), so each SM gets
 // about the same number of key tiles.  Every role walks the same item
@@ -88,21 +97,44 @@ struct Item {
   int qt, h0, nq, g, n;
   Span qs;
 };
+template <bool kViews>
 __device__ __forceinline__ Item item_of(int i, const MaskArgs& a) {
   const int pairs = a.per_group * a.Hkv;
-  const int rank = i / (pairs * a.n_seqs), rem = i % (pairs * a.n_seqs);
-  const int n = rem / pairs, pr = rem % pairs;
-  // Heaviest query tiles first: noisy query tile w and clean query tile
-  // n_qt / 2 + w both see w + 1 (or w + 2) key tiles, so the ranks take them
-  // in pairs from the last w down.
-  const int half = a.n_qt / 2, wq = half - 1 - rank / 2;
+  const int half = a.n_qt / 2;
   Item it;
-  it.qt = (rank & 1) ? wq : half + wq;
+  int pr;
+  if constexpr (!kViews) {
+    // Heaviest query tiles first: noisy query tile w and clean query tile
+    // n_qt / 2 + w both see w + 1 (or w + 2) key tiles, so the ranks take
+    // them in pairs from the last w down.
+    const int rank = i / (pairs * a.n_seqs), rem = i % (pairs * a.n_seqs);
+    const int wq = half - 1 - rank / 2;
+    it.n = rem / pairs;
+    pr = rem % pairs;
+    it.qt = (rank & 1) ? wq : half + wq;
+  } else {
+    // The same levels, each holding the clean items (one per sample and
+    // head pair, on the sample's first view) and then the noisy items (one
+    // per entry and head pair).
+    const int n_clean = pairs * a.n_samples, per_level = n_clean + pairs * a.n_seqs;
+    const int lvl = i / per_level;
+    int rem = i - lvl * per_level;
+    const int wq = half - 1 - lvl;
+    if (rem < n_clean) {
+      it.n = (rem / pairs) * a.views;
+      pr = rem % pairs;
+      it.qt = half + wq;
+    } else {
+      rem -= n_clean;
+      it.n = rem / pairs;
+      pr = rem % pairs;
+      it.qt = wq;
+    }
+  }
   it.g = pr / a.per_group;
   const int w = pr % a.per_group;
   it.h0 = it.g * a.G + 2 * w;                 // first head of the pair
   it.nq = (2 * w + 1 < a.G) ? 2 : 1;          // odd G: the last pair has one head
-  it.n = n;
   it.qs = span_of(it.qt, a.L, a.D);
   return it;
 }
@@ -138,6 +170,7 @@ __device__ __forceinline__ int vis_tile(const VisRanges& v, int j, int half) {
   return j < v.na ? v.a0 + j : half + (j - v.na);
 }
 
+template <bool kViews>
 __global__ void __launch_bounds__(kThreads, 1)
     mask_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -194,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; k * n_ctas < a.n_items && ok; ++k) {
       const int i = item_index(k, cta, n_ctas, a.n_items);
       if (i < 0) continue;
-      const Item it = item_of(i, a);
+      const Item it = item_of<kViews>(i, a);
       const int row_base = it.n * 2 * a.L;
       const VisRanges v = visible_ranges(it.qs, a);
       for (int j = 0; j < v.n; ++j) {
@@ -249,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int k = 0; k * n_ctas < a.n_items && ok; ++k) {
         const int i = item_index(k, cta, n_ctas, a.n_items);
         if (i < 0) continue;
-        const Item it = item_of(i, a);
+        const Item it = item_of<kViews>(i, a);
         const VisRanges v = visible_ranges(it.qs, a);
         if (v.n == 0) continue;
         if (!tc::mbar_wait(&q_full, kq & 1, a.status) || !tc::mbar_wait(&kv_full[st], ph, a.status)) {
@@ -318,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; k * n_ctas < a.n_items && ok; ++k) {
       const int ii = item_index(k, cta, n_ctas, a.n_items);
       if (ii < 0) continue;
-      const Item it = item_of(ii, a);
+      const Item it = item_of<kViews>(ii, a);
       if (t >= it.nq) continue;
       const int i = it.qt * kT + r;         // absolute row in [0, 2L)
       float m = -INFINITY, l = 0.f;
@@ -435,6 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_after();
       const int h = it.h0 + t;
       const int row = it.n * 2 * a.L + it.qt * kT + 32 * q;
+      // a clean tile's rows are the same in every view of its sample
+      const int n_out = kViews && it.qt >= a.n_qt / 2 ? a.views : 1;
       const float inv = 1.f / l;
       auto stage_box = [&](const uint32_t (&ov)[64]) {
 #pragma unroll
@@ -459,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::fence_proxy_async();
       __syncwarp();
       if (lane == 0) {
-        tc::tma_store_3d(&tm_out, stg, 0, h, row);
+        for (int vw = 0; vw < n_out; ++vw) tc::tma_store_3d(&tm_out, stg, 0, h, row + vw * 2 * a.L);
         tc::bulk_commit();
       }
       tc::tmem_ld_32x32b_x32(o_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
@@ -476,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::fence_proxy_async();
       __syncwarp();
       if (lane == 0) {
-        tc::tma_store_3d(&tm_out, stg, 64, h, row);
+        for (int vw = 0; vw < n_out; ++vw) tc::tma_store_3d(&tm_out, stg, 64, h, row + vw * 2 * a.L);
         tc::bulk_commit();
       }
       stored = true;
@@ -533,6 +568,13 @@ bool mask_attn_tc_supported(const bd_attn_shape& sh, int L) {
 cudaError_t launch_mask_attn_tc(const bd_attn_shape& sh, const void* q, const void* k,
                                 const void* v, void* out, int n_seqs, int L, int block,
                                 int32_t* status, cudaStream_t st) {
+  return launch_mask_attn_tc_views(sh, q, k, v, out, n_seqs, 1, L, block, status, st);
+}
+
+cudaError_t launch_mask_attn_tc_views(const bd_attn_shape& sh, const void* q, const void* k,
+                                      const void* v, void* out, int n_seqs, int views, int L,
+                                      int block, int32_t* status, cudaStream_t st) {
+  if (views <= 0 || n_seqs % views != 0) return cudaErrorInvalidValue;
   const int Hq = sh.n_heads_q, Hkv = sh.n_heads_kv;
   const uint64_t rows = static_cast<uint64_t>(n_seqs) * 2 * L;
   CUtensorMap tm_q, tm_k, tm_v, tm_out;
@@ -548,12 +590,17 @@ cudaError_t launch_mask_attn_tc(const bd_attn_shape& sh, const void* q, const vo
   a.n_qt = 2 * L / kT;
   a.out = static_cast<bf16*>(out);
   a.status = status;
-  cudaError_t e = cudaFuncSetAttribute(mask_attn_tc_kernel,
+  // views == 1: the plain kernel, without the shared-view bookkeeping
+  auto kern = views > 1 ? mask_attn_tc_kernel<true> : mask_attn_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   a.per_group = (a.G + 1) / 2;
   a.n_seqs = n_seqs;
-  const long long n_items = static_cast<long long>(a.n_qt) * n_seqs * a.per_group * Hkv;
+  a.views = views;
+  a.n_samples = n_seqs / views;
+  const long long n_items =
+      static_cast<long long>(a.n_qt / 2) * (n_seqs + a.n_samples) * a.per_group * Hkv;
   if (n_items <= 0 || n_items > (1LL << 30)) return cudaErrorInvalidValue;
   a.n_items = static_cast<int>(n_items);
   int sms = 0, dev = 0;
@@ -562,7 +609,7 @@ cudaError_t launch_mask_attn_tc(const bd_attn_shape& sh, const void* q, const vo
     sms = 148;
   // one persistent CTA per SM (one fits: 225 KB of shared memory, all of TMEM)
   const int grid = static_cast<int>(n_items < sms ? n_items : sms);
-  mask_attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, tm_out, a);
+  kern<<<grid, kThreads, kSmemBytes, st>>>(tm_q, tm_k, tm_v, tm_out, a);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -287,6 +287,28 @@ BD_API int bd_block_mask_attn(const bd_attn_shape* shape, const void* q,
                        const void* k, const void* v, void* out,
                        int32_t n_seqs, int32_t L, int32_t block, void* stream);
 
+/* bd_block_mask_attn_views -- bd_block_mask_attn for a batch whose entries
+ * come in groups of `views` consecutive entries that are views of one
+ * training sample ([N1] key design 2: the complementary masks m and 1 - m
+ * of one sample are two views of it, [N3]).  The views of a sample differ
+ * only in their noisy stream; their clean halves (rows L..2L-1 of q, k and
+ * v) must be equal, and the caller guarantees that.  A clean query sees
+ * clean keys only, so the clean rows of the output are equal across the
+ * views: the tensor-core path computes them once per sample, from its first
+ * view, and writes them into every view's rows (with views = 2 that is a
+ * quarter of the pairs of the plain call).  Arguments, layouts and errors as
+ * bd_block_mask_attn, plus:
+ *   views  >= 1 and dividing n_seqs (else BD_ERR_INVALID_ARG); views = 1 is
+ *          the plain call.
+ * If the clean halves of a sample's views differ, views other than the
+ * first receive the first view's clean rows.  Other shapes than the
+ * tensor-core kernel's (bf16, head_dim 128, L a multiple of 128) compute
+ * every view's rows from its own inputs. */
+BD_API int bd_block_mask_attn_views(const bd_attn_shape* shape, const void* q,
+                                    const void* k, const void* v, void* out,
+                                    int32_t n_seqs, int32_t views, int32_t L,
+                                    int32_t block, void* stream);
+
 /* bd_eval_exp2 -- diagnostic: the library's exponential approximations.
  *
  * No counterpart in the method: the attention softmax and the LM-head

@@ -378,6 +378,42 @@ def test_mask_attn_many_items_per_cta():
     assert float(np.abs(got - ref).max()) <= ATOL["bf16"]
 
 
+def _run_mask_views(cfg, t, views):
+    from decoding_bd_block_b200 import bd
+    from decoding_bd_block_b200.step import to_device
+    q, k, v = (to_device(t[x], cfg.dtype) for x in ("q", "k", "v"))
+    out = torch.full_like(q, float("nan"))
+    shape = bd.make_shape(cfg.n_heads_q, cfg.n_heads_kv, cfg.head_dim, cfg.dtype)
+    bd.bd_block_mask_attn_views(shape, q, k, v, out, cfg.n_seqs, views, cfg.L, cfg.block)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("L,D,dtype,d,Hq,Hkv,samples,views", [
+    (256, 32, "bf16", 128, 6, 2, 3, 4),   # tensor-core path, four views per sample
+    (384, 16, "bf16", 128, 4, 2, 2, 2),   # tensor-core path, many partly visible tiles
+    (96, 32, "f32", 64, 4, 2, 2, 2),      # CUDA-core path: every view computed from its inputs
+])
+def test_mask_attn_views_parity(L, D, dtype, d, Hq, Hkv, samples, views):
+    # Views of one sample share the clean stream (the generator writes the same
+    # x_0 rows into each view): the clean rows computed once per sample must be
+    # every view's, against the oracle run on each view on its own, and equal
+    # bit for bit to the plain call, which computes each view separately.
+    cfg = W.MaskAttnConfig(name="t", samples=samples, views=views, L=L, block=D, n_heads_q=Hq,
+                           n_heads_kv=Hkv, head_dim=d, seed=11, dtype=dtype)
+    t = W.make_mask_attn_inputs(cfg)
+    got = _run_mask_views(cfg, t, views)
+    ref = O.mask_attn(O.widen(t["q"], dtype), O.widen(t["k"], dtype), O.widen(t["v"], dtype), L, D)
+    assert float(np.abs(got - ref).max()) <= ATOL[dtype]
+    np.testing.assert_array_equal(got, _run_mask(cfg, t))
+
+
+def test_mask_attn_views_full_size_equals_plain_call():
+    cfg = W.MASK_ATTN
+    t = W.make_mask_attn_inputs(cfg)
+    np.testing.assert_array_equal(_run_mask_views(cfg, t, cfg.views), _run_mask(cfg, t))
+
+
 def test_mask_attn_full_size_sampled():
     cfg = W.MASK_ATTN
     t = W.make_mask_attn_inputs(cfg)

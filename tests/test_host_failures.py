@@ -153,3 +153,23 @@ def test_status_of_a_refused_call_launches_nothing(bd):
     assert bd._lib.bd_block_mask_attn(ctypes.byref(sh), None, FAKE, FAKE, FAKE, 1, 64, 32,
                                       None) == INVALID
     assert bd.bd_kernel_launches() == before
+
+
+def test_mask_attn_views_failures(bd):
+    # bd_block_mask_attn_views: views must be positive and divide n_seqs; the
+    # other checks are those of bd_block_mask_attn.  Nothing is launched.
+    before = bd.bd_kernel_launches()
+    sh = bd.make_shape(12, 2, 128, "bf16")
+
+    def call(q=FAKE, n_seqs=4, views=2, L=256, block=32, shape=sh):
+        return bd._lib.bd_block_mask_attn_views(ctypes.byref(shape), q, FAKE, FAKE, FAKE, n_seqs,
+                                                views, L, block, None)
+    assert call(views=0) == INVALID
+    assert call(views=-2) == INVALID
+    assert call(views=3) == INVALID           # 4 entries are not whole groups of 3
+    assert call(n_seqs=5) == INVALID
+    assert call(q=None) == INVALID
+    assert call(block=48) == INVALID          # block must divide L
+    assert call(L=48, block=16) == UNSUPPORTED  # L must be a multiple of 32
+    assert call(shape=bd.make_shape(12, 2, 96, "bf16")) == UNSUPPORTED
+    assert bd.bd_kernel_launches() == before
