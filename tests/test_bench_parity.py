@@ -40,3 +40,15 @@ def test_planted_mismatches_are_counted():
     assert not p["pass"]
     assert p["decision_mismatches"] == 1 and p["token_mismatches"] >= 1
     assert p["attn_max_abs_err"] >= 1.0 - 1e-6
+
+
+def test_mask_pair_counts_match_the_mask():
+    # The bench's algorithmic work for the 2L x 2L attention: its closed-form
+    # pair counts against a count of the oracle's mask.  Clean queries see no
+    # noisy key, which is why the views of one sample share their clean rows.
+    import oracle as O
+    for L, D in ((64, 8), (96, 32), (256, 32), (2048, 32)):
+        A = O.mixed_mask(L, D)
+        assert bench.mask_pairs(L, D) == int(A.sum())
+        assert bench.mask_clean_pairs(L, D) == int(A[L:].sum())
+        assert not A[L:, :L].any()
