@@ -7,6 +7,8 @@
  *        (papernotes.org), "Overall framework" and "Key designs" 1-4.
  *   [N2] Fast-dLLM (v1) article (senqingzn.com), "Core techniques" item 2,
  *        confidence-aware parallel decoding.
+ *   [N3] Fast-dLLM v2 abstract (hyper.ai, arXiv 2509.26328): training with
+ *        complementary masks.
  *   [N4] "Fast-dLLM v2: 2.5x inference speedup" (aigc.bar), "Acceleration
  *        engine" items 1 (hierarchical cache) and 2 (parallel decoding).
  *
