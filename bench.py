@@ -207,6 +207,20 @@ def measured_peaks():
     return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
 
 
+# Nominal per-GPU figures, for a second fraction beside the measured one:
+# HBM3e bandwidth (HGX B200) and dense bf16 tensor throughput.
+NOMINAL_PEAKS = {"GB/s": 7700.0, "TFLOP/s": 2250.0}
+
+
+def with_nominal(roofline: dict) -> dict:
+    """The roofline object with the fraction of the nominal peak of its unit
+    (the part's data-sheet figure) added beside the measured one."""
+    nom = NOMINAL_PEAKS.get(roofline.get("unit"))
+    if nom is not None and roofline.get("achieved") is not None:
+        roofline = dict(roofline, nominal_peak=nom, frac_of_nominal=roofline["achieved"] / nom)
+    return roofline
+
+
 def recorded_traffic(kernel: str):
     """DRAM bytes per launch from the committed ncu summary, if the kernel's
     source is unchanged since it was captured (else None)."""
@@ -687,6 +701,7 @@ def run_ours(args, cfg, tau, S, dist: Dist):
         line["cpu_baseline"], line["parity"] = cpu_baseline(
             cfg, a_in, s_in, tau, S, args.cpu_budget_s, None if step.active_only else got)
     if dist.rank == 0:
+        line["roofline"] = with_nominal(line["roofline"])
         print(json.dumps(line), flush=True)
 
 
@@ -835,6 +850,7 @@ def run_mask_attn(args, cfg, dist: Dist):
         "clocks": clocks,
     }
     if dist.rank == 0:
+        line["roofline"] = with_nominal(line["roofline"])
         print(json.dumps(line), flush=True)
 
 
@@ -908,6 +924,7 @@ def run_masked_ce(args, cfg, dist: Dist):
         "clocks": clocks,
     }
     if dist.rank == 0:
+        line["roofline"] = with_nominal(line["roofline"])
         print(json.dumps(line), flush=True)
 
 

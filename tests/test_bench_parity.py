@@ -52,3 +52,12 @@ def test_mask_pair_counts_match_the_mask():
         assert bench.mask_pairs(L, D) == int(A.sum())
         assert bench.mask_clean_pairs(L, D) == int(A[L:].sum())
         assert not A[L:, :L].any()
+
+
+def test_nominal_fraction_beside_the_measured_one():
+    r = bench.with_nominal({"unit": "GB/s", "achieved": 3850.0, "peak": 6545.0, "frac": 0.588})
+    assert r["nominal_peak"] == 7700.0 and abs(r["frac_of_nominal"] - 0.5) < 1e-12
+    assert r["frac"] == 0.588  # the measured-peak fraction is left as it is
+    t = bench.with_nominal({"unit": "TFLOP/s", "achieved": 1125.0})
+    assert abs(t["frac_of_nominal"] - 0.5) < 1e-12
+    assert "frac_of_nominal" not in bench.with_nominal({"unit": "x/s", "achieved": 1.0})
